@@ -1,0 +1,395 @@
+"""Benchmark of the CSA2 decode step over an FP4 global KV cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one decode token through the decoder's 20-layer CSA2 schedule (first group
+Full + 3 Reuse, the Full layer building the 2048 x 8 candidate pool; then 4 groups of
+Reindex + 3 Reuse), preceded by the append of the token's own compressed entry.  The
+default workload is that step at a context of 131,072 entries (64 heads x 512, indexer
+16 x 128, Top-512, window 128, 1% outlier rows); ``--workload decoder_step_1m`` runs it at
+1,048,576.  The metric is decode layer-steps/s (20 per step) over the whole job.
+
+Timing: W untimed warm-up steps, then K steps, each replayed from CUDA graphs and timed
+with CUDA events on the launching stream; L2 is flushed (a 256 MB write) between steps,
+outside the timed events.  Multi-GPU: one independent replica per rank (the decode step of
+one sequence does not shard), max time over ranks.  rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s at 128K and 1M ctx; achieved HBM GB/s vs roofline"
+UNIT = "layer-steps/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"csa2_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of the same workload
+# ----------------------------------------------------------------------------------------
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(W, budget_s: float):
+    """Run the oracle over the decoder schedule for the workload's query, step after step,
+    until ``budget_s`` seconds of oracle work.  The stored FP4 cache is the oracle's own
+    quantisation of the seeded rows, filled on first touch outside the timed spans (the GPU's
+    cache is likewise filled before timing); each timed step quantises the appended row,
+    scores, selects, builds the pool, re-scores the pool, dequantises the selected rows and
+    attends.  Returns (layer_steps, seconds, description)."""
+    from fp4_kv_cache_03_b200 import synth
+    from oracle import csa2_ref as R
+    n = W.lengths[0]
+    kI = synth.bf16_bits_to_f32(synth.index_k_rows(W.seed, 0, n, W.d_I)).astype(np.float64)
+    kv = synth.kv_rows(W.seed, 0, n, W.D, W.outlier_frac)
+    x_new = synth.append_rows(W.seed, 0, 1, W.D)
+    kv[n - 1] = x_new[0]
+    kI[n - 1] = synth.bf16_bits_to_f32(synth.append_index_k(W.seed, 0, 1, W.d_I))[0]
+    stored = {}                                    # row -> (codes, scales): the FP4 cache
+
+    def fill(pos):
+        need = [int(p) for p in pos if int(p) not in stored]
+        if need:
+            c, sc = R.quantize_rows(kv[need])
+            for i, p in enumerate(need):
+                stored[p] = (c[i], sc[i])
+
+    t_q = int(W.q_pos()[0])
+    layers = []
+    for li, mode in enumerate(W.modes):
+        q = synth.bf16_bits_to_f32(synth.queries(W.seed, li, 1, W.H, W.D))[0]
+        qI = synth.bf16_bits_to_f32(synth.index_queries(W.seed, li, 1, W.H_I, W.d_I))[0]
+        w = synth.index_weights(W.seed, li, 1, W.H_I)[0]
+        pos = R.window_positions(t_q, W.window)
+        swa = synth.bf16_bits_to_f32(synth.swa_rows(W.seed, li, 0, int(pos[0]), len(pos), W.D))
+        layers.append((mode, q, qI, w, swa))
+    done, t_total, steps = 0, 0.0, 0
+    while True:
+        t0 = time.perf_counter()
+        untimed = 0.0
+        R.quantize_rows(x_new)                                   # a1 append
+        latest = pool = None
+        for mode, q, qI, w, swa in layers:
+            if mode == "full":
+                sc = R.index_scores(qI, w, kI)
+                latest = R.topk_ascending(sc, W.topk)
+                if W.pool_blocks and pool is None:
+                    pool = R.build_pool(sc, W.pool_blocks, W.block)
+            elif mode == "reindex":
+                latest = R.reindex(qI, w, kI, pool, W.block, n, W.topk)
+            sel = latest[latest >= 0]
+            t1 = time.perf_counter()
+            fill(sel)
+            untimed += time.perf_counter() - t1
+            rows = R.dequantize_rows(np.stack([stored[int(p)][0] for p in sel]),
+                                     np.stack([stored[int(p)][1] for p in sel]))
+            R.sparse_attention(q, rows, swa, 1.0 / math.sqrt(W.D))
+            done += 1
+        t_total += time.perf_counter() - t0 - untimed
+        steps += 1
+        if t_total >= budget_s:
+            break
+    return done, t_total, (f"{steps} decoder step(s) x {len(W.modes)} layers, 1 query, "
+                           f"{n} entries; cache quantised outside the timed spans")
+
+
+# ----------------------------------------------------------------------------------------
+def run_reference(args, rank):
+    """The oracle arm: the same metric, on the host cores, bounded."""
+    if rank != 0:
+        return
+    from fp4_kv_cache_03_b200 import synth
+    W = synth.workload(args.workload)
+    ls, t, what = oracle_sample(W, max(10.0, 2.0 * args.steps))
+    v = ls / t
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t * len(W.modes) / ls,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": W.name, "context_entries": W.lengths[0],
+                                            "layers": len(W.modes), "batch": W.num_q},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": what},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from fp4_kv_cache_03_b200 import csa2, synth
+    from fp4_kv_cache_03_b200.workload import DeviceWorkload
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    W = synth.workload(args.workload)
+    dw = DeviceWorkload(W, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    n_layers = len(W.modes)
+    n_index = sum(1 for m in W.modes if m != synth.REUSE)
+
+    # --- capture the step as three graphs: append | Full index | the rest ---
+    def part_append():
+        dw.append(stream=stream)
+
+    full_li = W.modes.index(synth.FULL)
+
+    def part_full():
+        L = dw.layers[full_li]
+        csa2.index_full(L.qI, L.w, dw.idx_k, dw.seqs, W.topk, dw.indices[0], dw.ws_full,
+                        dw.max_visible, q_visible=dw.q_visible, pool_blocks=W.pool_blocks,
+                        block=W.block, pool=dw.pool if W.pool_blocks else None, stream=stream)
+
+    def part_rest():
+        latest, n_idx = dw.indices[0], 1
+        for li, L in enumerate(dw.layers):
+            if L.mode == synth.REINDEX:
+                idx = dw.indices[n_idx]
+                n_idx += 1
+                csa2.index_pool(L.qI, L.w, dw.idx_k, dw.seqs, dw.pool, W.pool_blocks, W.block,
+                                W.topk, idx, dw.ws_pool, q_visible=dw.q_visible, stream=stream)
+                latest = idx
+            elif L.mode == synth.FULL and li != full_li:
+                raise NotImplementedError("one Full layer per step")
+            csa2.sparse_attn(L.q, dw.kv_codes, dw.kv_scales, dw.seqs, latest, L.swa, L.swa_start,
+                             dw.q_pos, W.window, dw.scale, dw.out[li], dw.ws_attn, lse=dw.lse[li],
+                             stream=stream)
+
+    graphs = []
+    with torch.cuda.stream(stream):
+        for fn in (part_append, part_full, part_rest):   # eager once before capture
+            fn()
+        stream.synchronize()
+        for fn in (part_append, part_full, part_rest):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+    stream.synchronize()
+    st = dw.status()
+    if st != csa2.OK:
+        raise csa2.CSA2Error(st, "warm-up step")
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def one_step(ev):
+        ev[0].record(stream)
+        graphs[0].replay()
+        ev[1].record(stream)
+        graphs[1].replay()
+        ev[2].record(stream)
+        graphs[2].replay()
+        ev[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    stream.synchronize()
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    props = torch.cuda.get_device_properties(local_rank)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else local_rank)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            flush.zero_()
+            one_step(evs[k])
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    full_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    t_total = sum(step_ms) / 1e3
+    if world > 1:
+        t = torch.tensor([t_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_total = float(t.item())
+    st = dw.status()
+    if st != csa2.OK:
+        raise csa2.CSA2Error(st, "timed steps")
+
+    # --- e2e through the API with host buffers: inputs H2D each step, results D2H ---
+    pin = lambda t: t.detach().cpu().pin_memory()
+    h_in = [(pin(dw.append_x), dw.append_x), (pin(dw.append_k), dw.append_k)]
+    for L in dw.layers:
+        h_in.append((pin(L.q), L.q))
+        h_in.append((pin(L.swa[-1:]), L.swa[-1:]))      # the step's new window row
+        if L.qI is not None:
+            h_in += [(pin(L.qI), L.qI), (pin(L.w), L.w)]
+    h_out = [(torch.empty_like(o, device="cpu").pin_memory(), o) for o in dw.out]
+    h2d = sum(h.numel() * h.element_size() for h, _ in h_in)
+    d2h = sum(h.numel() * h.element_size() for h, _ in h_out)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            flush.zero_()
+            e2e_ev[k][0].record(stream)
+            for h, d in h_in:
+                d.copy_(h, non_blocking=True)
+            for g in graphs:
+                g.replay()
+            for h, d in h_out:
+                h.copy_(d, non_blocking=True)
+            e2e_ev[k][1].record(stream)
+    stream.synchronize()
+    e2e_t = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_t = float(t.item())
+
+    # --- roofline of the dominant op: the Full-mode index (score scan + Top-K + pool) ---
+    hbm, tflops, src = peaks()
+    n_ctx = W.lengths[0]
+    alg_bytes = n_ctx * W.d_I * 2                  # the indexer-K stream, 256 B per entry
+    full_s = statistics.mean(full_ms) / 1e3
+    achieved = alg_bytes / full_s / 1e9
+    steps_total = args.steps * world
+    value = steps_total * n_layers / t_total
+    launches_per_step = (1 if W.append else 0) + 6 * n_index + 2 * n_layers
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp4->fp32",
+        "data": "synthetic (seeded; shapes of the pages' decoder, no weights)",
+        "config": {"workload": W.name, "context_entries": n_ctx, "layers": n_layers,
+                   "schedule": "Full+pool, 3 Reuse, 4x(Reindex + 3 Reuse)", "batch": W.num_q,
+                   "D": W.D, "H": W.H, "indexer": f"{W.H_I}x{W.d_I}", "topk": W.topk,
+                   "window": W.window, "pool": f"{W.pool_blocks}x{W.block}",
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "csa2_index_full (score scan + Top-K + pool select)",
+                     "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+                     "alg_bytes_per_launch": alg_bytes, "ms_per_launch": full_s * 1e3},
+        "e2e": {"value": steps_total * n_layers / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ls, t, what = oracle_sample(W, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": ls / t, "unit": UNIT, "cores": cpu_threads(),
+                                "kind": "oracle", "sample": what}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decoder_step_128k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

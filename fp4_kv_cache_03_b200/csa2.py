@@ -1,0 +1,190 @@
+"""ctypes binding of libcsa2.so (the C ABI in include/csa2.h).
+
+Argument marshalling only: every step of the CSA2 path runs in the library's CUDA
+kernels.  Tensors are PyTorch tensors (device memory and streams are PyTorch's);
+each function passes their pointers to the C entry point of the same name and
+raises ``CSA2Error`` on a non-OK status.  If the library is not built, importing
+anything that needs it raises -- there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_float, c_int32, c_int64, c_size_t, c_void_p
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcsa2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT = range(6)
+MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
+STATUS_BYTES = 256
+
+
+class CSA2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class Seqs(ctypes.Structure):
+    """csa2_seqs_t: ragged batch description (device arrays)."""
+    _fields_ = [("num_seqs", c_int32), ("q_per_seq", c_int32),
+                ("seq_start", c_void_p), ("seq_len", c_void_p)]
+
+
+_lib = None
+
+_SIGS = {
+    "csa2_quant_append_workspace": (c_size_t, []),
+    "csa2_quant_append": (c_int32, [c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                    c_int64, c_void_p, c_void_p, c_int32, c_void_p, c_size_t,
+                                    c_void_p]),
+    "csa2_index_full_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
+    "csa2_index_full": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                  c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p, c_int32,
+                                  c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa2_index_pool_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32]),
+    "csa2_index_pool": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                  c_int64, Seqs, c_void_p, c_void_p, c_int32, c_int32, c_int32,
+                                  c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa2_sparse_attn_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
+    "csa2_sparse_attn": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                   c_int64, Seqs, c_void_p, c_int32, c_void_p, c_int64, c_void_p,
+                                   c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
+                                   c_size_t, c_void_p]),
+    "csa2_status_reset": (c_int32, [c_void_p, c_void_p]),
+    "csa2_status_fetch": (c_int32, [c_void_p, c_void_p]),
+    "csa2_status_string": (ctypes.c_char_p, [c_int32]),
+    "csa2_device_sms": (c_int32, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcsa2.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m fp4_kv_cache_03_b200.build_lib`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().csa2_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise CSA2Error(status, what)
+
+
+def _p(t) -> c_void_p | None:
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to libcsa2 must be contiguous"
+    return c_void_p(t.data_ptr())
+
+
+def _s(stream) -> c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_void_p(stream.cuda_stream)
+
+
+def _u16(t):
+    """bf16 tensors travel as their 16-bit patterns."""
+    if t is None:
+        return None
+    assert t.dtype in (torch.bfloat16, torch.uint16, torch.int16), t.dtype
+    return _p(t)
+
+
+def make_seqs(seq_start: torch.Tensor, seq_len: torch.Tensor, q_per_seq: int = 1) -> Seqs:
+    assert seq_start.dtype == torch.int64 and seq_len.dtype == torch.int32
+    s = Seqs(int(seq_start.numel()), int(q_per_seq), _p(seq_start), _p(seq_len))
+    s._keep = (seq_start, seq_len)  # keep the tensors alive with the struct
+    return s
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed byte workspace (its status word starts clear)."""
+    return torch.zeros(max(int(nbytes), STATUS_BYTES), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------------------------
+# entry points
+# ------------------------------------------------------------------------------------
+def quant_append_workspace() -> int:
+    return int(lib().csa2_quant_append_workspace())
+
+
+def quant_append(x, dst_row, kv_codes, kv_scales, ws, idx_k_in=None, idx_k=None, stream=None):
+    assert x.dtype == torch.float32 and dst_row.dtype == torch.int64
+    rows, D = x.shape
+    d_I = idx_k.shape[1] if idx_k is not None else 0
+    _check(lib().csa2_quant_append(_p(x), rows, D, _p(dst_row), _p(kv_codes), _p(kv_scales),
+                                   kv_codes.shape[0], _u16(idx_k_in), _u16(idx_k), d_I, _p(ws),
+                                   ws.numel(), _s(stream)), "csa2_quant_append")
+
+
+def index_full_workspace(num_q, max_visible, topk, pool_blocks=0, block=8) -> int:
+    return int(lib().csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks, block))
+
+
+def index_full(qI, w, idx_k, seqs: Seqs, topk, indices, ws, max_visible, q_visible=None,
+               pool_blocks=0, block=8, pool=None, stream=None):
+    num_q, H_I, d_I = qI.shape
+    assert w.dtype == torch.float32 and indices.dtype == torch.int32
+    _check(lib().csa2_index_full(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
+                                 seqs, _p(q_visible), int(max_visible), topk, _p(indices),
+                                 pool_blocks, block, _p(pool), _p(ws), ws.numel(), _s(stream)),
+           "csa2_index_full")
+
+
+def index_pool_workspace(num_q, pool_blocks, block, topk) -> int:
+    return int(lib().csa2_index_pool_workspace(num_q, pool_blocks, block, topk))
+
+
+def index_pool(qI, w, idx_k, seqs: Seqs, pool, pool_blocks, block, topk, indices, ws,
+               q_visible=None, stream=None):
+    num_q, H_I, d_I = qI.shape
+    _check(lib().csa2_index_pool(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
+                                 seqs, _p(q_visible), _p(pool), pool_blocks, block, topk,
+                                 _p(indices), _p(ws), ws.numel(), _s(stream)),
+           "csa2_index_pool")
+
+
+def sparse_attn_workspace(num_q, H, D, topk, window) -> int:
+    return int(lib().csa2_sparse_attn_workspace(num_q, H, D, topk, window))
+
+
+def sparse_attn(q, kv_codes, kv_scales, seqs: Seqs, indices, swa_kv, swa_start, q_pos, window,
+                softmax_scale, out, ws, lse=None, stream=None):
+    num_q, H, D = q.shape
+    topk = indices.shape[1] if indices is not None else 0
+    assert out.dtype == torch.float32 and q_pos.dtype == torch.int64
+    _check(lib().csa2_sparse_attn(_u16(q), num_q, H, D, _p(kv_codes), _p(kv_scales),
+                                  kv_codes.shape[0], seqs, _p(indices), topk, _u16(swa_kv),
+                                  swa_kv.shape[0] if swa_kv is not None else 0, _p(swa_start),
+                                  _p(q_pos), window, float(softmax_scale), _p(out), _p(lse),
+                                  _p(ws), ws.numel(), _s(stream)), "csa2_sparse_attn")
+
+
+def status_reset(ws, stream=None) -> None:
+    _check(lib().csa2_status_reset(_p(ws), _s(stream)), "csa2_status_reset")
+
+
+def status_fetch(ws, stream=None) -> int:
+    """Wait for the stream; return the status word recorded in ``ws`` (0 = OK)."""
+    return int(lib().csa2_status_fetch(_p(ws), _s(stream)))
+
+
+def device_sms() -> int:
+    return int(lib().csa2_device_sms())

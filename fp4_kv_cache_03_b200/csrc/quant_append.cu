@@ -1,0 +1,112 @@
+// a1: quantise main-KV rows to FP4 (E2M1 codes + one E4M3 scale per 16 channels, no
+// global scale) and append them to the cache; optionally copy the indexer-K row too.
+// Format: aprilzz.com "DeepSeek V4.1 Flash 发布…", section "FP4 KV 与部署层的几个改动";
+// gkm0120.cn "技术调研报告" §2.2.1.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+namespace {
+
+// E2M1 magnitude code of q >= 0: nearest of {0,.5,1,1.5,2,3,4,6}, exact midpoints to the
+// even code, saturating at 6.  Each comparison is one threshold of the grid.
+__device__ __forceinline__ uint32_t e2m1_magnitude(float q) {
+  return (uint32_t)(q > 0.25f) + (uint32_t)(q >= 0.75f) + (uint32_t)(q > 1.25f) +
+         (uint32_t)(q >= 1.75f) + (uint32_t)(q > 2.5f) + (uint32_t)(q >= 3.5f) +
+         (uint32_t)(q > 5.0f);
+}
+
+// value of a non-negative E4M3 code (bias 7; exponent field 0 is subnormal m * 2^-9)
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  if (e == 0) return (float)m * 0.001953125f;
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+__global__ void __launch_bounds__(256) quant_append_kernel(
+    const float* __restrict__ x, int rows, int D, const int64_t* __restrict__ dst_row,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int64_t cap,
+    const uint16_t* __restrict__ kin, uint16_t* __restrict__ kout, int d_I, int* status) {
+  const int gpr = D >> 4;                      // channel groups per row
+  const int cpr = kin ? (d_I >> 3) : 0;        // 16-byte chunks of indexer K per row
+  const int64_t n_q = (int64_t)rows * gpr;
+  const int64_t n_c = (int64_t)rows * cpr;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+
+  if (gid < n_q) {
+    const int r = (int)(gid / gpr), g = (int)(gid % gpr);
+    const int64_t dst = dst_row[r];
+    if (dst < 0 || dst >= cap) {
+      report(status, CSA2_ERR_CAPACITY);
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(x + (int64_t)r * D + g * 16);
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 t = __ldg(src + i);
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      const __nv_fp8_storage_t sc =
+          __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+      const float s = e4m3_value((uint32_t)sc & 0x7Fu);
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t sign = __float_as_uint(v[i]) >> 31;
+        const uint32_t mag = (s != 0.0f) ? e2m1_magnitude(__fdiv_rn(fabsf(v[i]), s)) : 0u;
+        packed[i >> 3] |= ((sign << 3) | mag) << (4 * (i & 7));
+      }
+      uint2* dc = reinterpret_cast<uint2*>(codes + dst * (int64_t)(D >> 1) + g * 8);
+      *dc = make_uint2(packed[0], packed[1]);
+      scales[dst * (int64_t)gpr + g] = (uint8_t)sc;
+    }
+  }
+  if (gid < n_c) {
+    const int r = (int)(gid / cpr), c = (int)(gid % cpr);
+    const int64_t dst = dst_row[r];
+    if (dst >= 0 && dst < cap) {
+      const uint4 t = __ldg(reinterpret_cast<const uint4*>(kin + (int64_t)r * d_I) + c);
+      reinterpret_cast<uint4*>(kout + dst * (int64_t)d_I)[c] = t;
+    } else {
+      report(status, CSA2_ERR_CAPACITY);
+    }
+  }
+}
+
+}  // namespace
+}  // namespace csa2
+
+extern "C" size_t csa2_quant_append_workspace(void) { return CSA2_STATUS_BYTES; }
+
+extern "C" csa2_status_t csa2_quant_append(const float* x, int32_t rows, int32_t D,
+                                           const int64_t* dst_row, uint8_t* kv_codes,
+                                           uint8_t* kv_scales, int64_t cap_rows,
+                                           const uint16_t* idx_k_in, uint16_t* idx_k,
+                                           int32_t d_I, void* workspace, size_t ws_bytes,
+                                           void* stream) {
+  if (rows < 0 || D < 32 || D > 4096 || (D % 32) != 0 || cap_rows <= 0) return CSA2_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < CSA2_STATUS_BYTES) return CSA2_ERR_CAPACITY;
+  if (rows == 0) return CSA2_OK;
+  if (!x || !dst_row || !kv_codes || !kv_scales) return CSA2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 7))
+    return CSA2_ERR_INVALID_ARG;
+  if (idx_k_in) {
+    if (!idx_k || d_I < 8 || (d_I % 8) != 0) return CSA2_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(idx_k_in) & 15) || (reinterpret_cast<uintptr_t>(idx_k) & 15))
+      return CSA2_ERR_INVALID_ARG;
+  }
+  const int64_t nq = (int64_t)rows * (D / 16);
+  const int64_t nc = idx_k_in ? (int64_t)rows * (d_I / 8) : 0;
+  const int64_t n = nq > nc ? nq : nc;
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  if (blocks > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;
+  csa2::quant_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+      x, rows, D, dst_row, kv_codes, kv_scales, cap_rows, idx_k_in, idx_k, idx_k_in ? d_I : 0,
+      static_cast<int*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}

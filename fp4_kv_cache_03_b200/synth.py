@@ -104,10 +104,11 @@ def index_weights(seed: int, layer: int, num_q: int, H_I: int,
     return r.integers(lo, hi + 1, size=(num_q, H_I)).astype(np.float32)
 
 
-def swa_rows(seed: int, layer: int, start: int, count: int, D: int) -> np.ndarray:
-    """Sliding-window KV rows of one layer, bf16 N(0,1) bits, row r = token position r."""
+def swa_rows(seed: int, layer: int, seq: int, start: int, count: int, D: int) -> np.ndarray:
+    """Sliding-window KV rows of one layer and sequence, bf16 N(0,1) bits; row r of the
+    result is token position start + r."""
     def blk(b):
-        r = _rng(seed, S_SWA, layer, D, b)
+        r = _rng(seed, S_SWA, layer, seq, D, b)
         return f32_to_bf16_bits(r.standard_normal((ROW_BLOCK, D), dtype=np.float32))
     return _blocked(blk, start, count, D, np.uint16)
 

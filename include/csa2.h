@@ -1,0 +1,207 @@
+/*
+ * csa2.h -- C ABI of the CSA2 attention step over an FP4 global KV cache (B200, sm_100a).
+ *
+ * What is computed follows the DeepSeek-V4.1-Flash pages:
+ *   [MTP]  aprilzz.com "DeepSeek V4.1 Flash 发布：KV cache 降到 890 字节/token…",
+ *          sections "CSA2：在层的维度上共享缓存" (Full / Reindex / Reuse, Top-512, the
+ *          2048 x 8 candidate pool), "FP4 KV 与部署层的几个改动" (E2M1 values, one E4M3
+ *          scale per 16 channels, no global scale), "把 prefill 砍掉一半" (128-token window)
+ *   [SURV] gkm0120.cn "DeepSeek-V4.1-Flash 技术调研报告", §2.2.2 (modes table) and
+ *          §2.2.3 (hierarchical sparse indexer)
+ *   [OVR]  "DeepSeek-V4.1-Flash：推动 KV 缓存压缩极限", 摘要 (FP4 KV + cross-layer reuse)
+ * Details the pages leave open are fixed as stated at each entry point.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers marked "device" are CUDA device pointers; "host" values are plain
+ *     integers.  The caller owns every buffer; the library allocates nothing and keeps
+ *     no state between calls.
+ *   - bf16 data is passed as its raw 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *     enqueues work on it and returns; results are ready when the stream is.
+ *   - Shape, pointer and workspace-size errors are detected on the host and returned
+ *     before anything is enqueued.  Values that live in device memory (lengths, row
+ *     ids, indices) are checked by the kernels: a bad value is skipped and the first
+ *     such error is recorded in the status word at the start of `workspace`, which
+ *     csa2_status_fetch() returns.  Kernels never trap; every wait inside a kernel is
+ *     bounded and reports CSA2_ERR_TIMEOUT when its bound runs out.
+ *   - `workspace` is caller-allocated device memory of at least the size the matching
+ *     *_workspace() function returns, 256-byte aligned.  Its first CSA2_STATUS_BYTES
+ *     hold the sticky status word: clear it once with csa2_status_reset(); calls never
+ *     clear it.  Two calls that overlap on the GPU must not share a workspace.
+ *   - Launch failures map to CSA2_ERR_CUDA.
+ *
+ * Cache layout in HBM (row-major, one row per compressed entry)
+ *   kv_codes  uint8 [cap_rows][D/2]   E2M1 codes, byte k = code[2k] | code[2k+1] << 4
+ *   kv_scales uint8 [cap_rows][D/16]  E4M3 scale of channels 16g .. 16g+15
+ *   idx_k     bf16  [cap_rows][d_I]   indexer keys
+ *   That is 9D/16 bytes of main KV per entry: 288 B at D = 512.
+ *   Sequence s owns rows [seq_start[s], seq_start[s] + seq_len[s]); a position p of
+ *   the sequence is row seq_start[s] + p.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Static per-layer mode ([SURV] §2.2.2, [MTP] "CSA2：…"):
+ *   FULL    - own indexer over every visible entry, new Top-K (the decoder's first Full
+ *             layer also builds the candidate pool);
+ *   REINDEX - reuses main KV and indexer K, scores only the pool with its own indexer Q;
+ *   REUSE   - no indexer; attends with the latest Full/Reindex indices. */
+typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode_t;
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_INVALID_ARG = 1,  /* bad shape / pointer, or a device-side value out of range */
+  CSA2_ERR_UNSUPPORTED = 2,  /* a shape this build has no kernel for */
+  CSA2_ERR_CAPACITY = 3,     /* workspace too small, or a row outside the cache */
+  CSA2_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  CSA2_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel ran out */
+} csa2_status_t;
+
+#define CSA2_STATUS_BYTES 256
+
+/* Ragged batch description.  Query q belongs to sequence q / q_per_seq. */
+typedef struct {
+  int32_t num_seqs;           /* host: number of sequences (>= 1) */
+  int32_t q_per_seq;          /* host: queries per sequence (decode: 1) */
+  const int64_t* seq_start;   /* device [num_seqs]: cache row of position 0 */
+  const int32_t* seq_len;     /* device [num_seqs]: entries stored for the sequence */
+} csa2_seqs_t;
+
+/* ---------------------------------------------------------------------------------
+ * a1. Quantise + append main-KV rows ([MTP] "FP4 KV 与部署层的几个改动": E2M1 values with
+ * one E4M3 scale per 16 channels, no global scale).  For each row r and channel group g:
+ *   amax  = max |x[r][16g .. 16g+15]|
+ *   scale = E4M3(amax / 6)                  fp32 divide, round-to-nearest-even, saturate
+ *   code  = E2M1(x / dec(scale))            fp32 divide, RNE, saturate to +-6, sign kept;
+ *                                           a zero scale gives signed-zero codes
+ * and writes codes/scale into cache row dst_row[r].  If idx_k_in is not NULL, its row r
+ * (d_I bf16) is copied to idx_k row dst_row[r] as well.
+ *   x         device fp32 [rows][D]          D a multiple of 32, 32 <= D <= 4096
+ *   dst_row   device int64 [rows]            must be in [0, cap_rows): else skipped and
+ *                                            CSA2_ERR_CAPACITY is recorded
+ *   kv_codes, kv_scales  device, layout above, cap_rows rows
+ *   idx_k_in  device bf16 [rows][d_I] or NULL;  idx_k device bf16 [cap_rows][d_I]
+ *   workspace >= csa2_quant_append_workspace() bytes (status word only)
+ * rows = 0 is a no-op. */
+CSA2_API size_t csa2_quant_append_workspace(void);
+CSA2_API csa2_status_t csa2_quant_append(const float* x, int32_t rows, int32_t D, const int64_t* dst_row,
+                                uint8_t* kv_codes, uint8_t* kv_scales, int64_t cap_rows,
+                                const uint16_t* idx_k_in, uint16_t* idx_k, int32_t d_I,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a2 + a3 (+ a4).  Full-mode indexer ([MTP] "CSA2：…": Full selects a new Top-512;
+ * [SURV] §2.2.3: the decoder's first Full layer bounds the search of deeper layers).
+ * For query q of sequence s with visible entries V = q_visible[q] (seq_len[s] if
+ * q_visible is NULL), and every position e < V:
+ *   score[q][e] = sum_h w[q][h] * max(0, sum_d qI[q][h][d] * idx_k[seq_start[s]+e][d])
+ * (bf16 inputs, fp32 tensor-core accumulation: exact for the integer-valued inputs the
+ * tests use).  indices[q][*] = the topk positions ranked first by (score desc, position
+ * asc), written in ascending position order, padded with -1 when V < topk.
+ * If pool_blocks > 0 it also builds the candidate pool: block j covers positions
+ * [block*j, block*j + block) below V, its score is the max of their scores, and
+ * pool[q][*] = the pool_blocks block ids ranked first by (block score desc, id asc),
+ * ascending, -1 padded.
+ *   qI        device bf16 [num_q][H_I][d_I]      1 <= H_I <= 32, d_I in {64, 128}
+ *   w         device fp32 [num_q][H_I]
+ *   idx_k     device bf16 [cap_rows][d_I], base 16-byte aligned, cap_rows < 2^31
+ *   q_visible device int32 [num_q] or NULL; values above seq_len are clamped and
+ *             CSA2_ERR_INVALID_ARG is recorded
+ *   max_visible host bound on every V (sizes the workspace); larger V are clamped and
+ *             CSA2_ERR_CAPACITY is recorded
+ *   topk      1 <= topk <= 4096;  indices device int32 [num_q][topk]
+ *   pool_blocks 0 or 1..8192; block a power of two in 1..32 (the pages use 8);
+ *             pool device int32 [num_q][pool_blocks] (may be NULL when pool_blocks = 0)
+ *   workspace >= csa2_index_full_workspace(...) bytes */
+CSA2_API size_t csa2_index_full_workspace(int32_t num_q, int32_t max_visible, int32_t topk,
+                                 int32_t pool_blocks, int32_t block);
+CSA2_API csa2_status_t csa2_index_full(const uint16_t* qI, const float* w, int32_t num_q, int32_t H_I,
+                              int32_t d_I, const uint16_t* idx_k, int64_t cap_rows,
+                              csa2_seqs_t seqs, const int32_t* q_visible, int32_t max_visible,
+                              int32_t topk, int32_t* indices,
+                              int32_t pool_blocks, int32_t block, int32_t* pool,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a5. Reindex over the pool ([SURV] §2.2.2: Reindex reuses main KV and indexer K but has
+ * its own indexer Q and re-selects; [MTP] "CSA2：…": Reindex layers only score inside the
+ * bounded pool).  Candidates of query q: positions block*pool[q][i] + r, r < block, for
+ * every pool entry >= 0, that are below V.  Each is scored with this layer's qI/w as in
+ * csa2_index_full; indices[q][*] = the topk candidates ranked first by (score desc,
+ * position asc), ascending, -1 padded.  pool must list block ids in ascending order
+ * followed by -1 padding, as csa2_index_full writes it.
+ *   block must be 8 (the pages' block size); pool_blocks 1..8192; other arguments as
+ *   csa2_index_full. */
+CSA2_API size_t csa2_index_pool_workspace(int32_t num_q, int32_t pool_blocks, int32_t block,
+                                 int32_t topk);
+CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32_t num_q, int32_t H_I,
+                              int32_t d_I, const uint16_t* idx_k, int64_t cap_rows,
+                              csa2_seqs_t seqs, const int32_t* q_visible,
+                              const int32_t* pool, int32_t pool_blocks, int32_t block,
+                              int32_t topk, int32_t* indices,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a7. Sparse attention with the joint sliding window ([MTP] "把 prefill 砍掉一半": every
+ * layer keeps a 128-token window; "CSA2：…": each layer keeps its own main Q and window
+ * KV).  For query q of sequence s at token position t = q_pos[q], the key/value rows are
+ *   - for every i with p = indices[q][i] >= 0: the dequantised cache row seq_start[s] + p
+ *     (e2m1(code) * e4m3(scale), exact in bf16); p >= seq_len[s] is skipped and
+ *     CSA2_ERR_INVALID_ARG recorded;
+ *   - the window: swa_kv rows swa_start[s] + u for token positions
+ *     u = max(0, t - window + 1) .. t (rows outside [0, swa_rows) are skipped and
+ *     CSA2_ERR_CAPACITY recorded).
+ * Keys equal values (one vector per row).  Per head h:
+ *   l_j = softmax_scale * q[q][h] . row_j;  out[q][h] = sum_j softmax(l)_j row_j;
+ *   lse[q][h] = log(sum_j exp(l_j)) (natural log); no rows at all gives out = 0,
+ *   lse = -inf.  The two sets share one softmax; a row in both counts twice.
+ *   q         device bf16 [num_q][H][D]        H a multiple of 16 in 16..128, D a power of
+ *             two in 32..512 (other shapes return CSA2_ERR_UNSUPPORTED)
+ *   indices   device int32 [num_q][topk]       0 <= topk <= 2048
+ *   swa_kv    device bf16 [swa_rows][D];  swa_start device int64 [num_seqs] (may be
+ *             negative: only rows of window positions are read)
+ *   q_pos     device int64 [num_q]
+ *   window    0 .. 1024
+ *   out       device fp32 [num_q][H][D];  lse device fp32 [num_q][H] or NULL
+ *   workspace >= csa2_sparse_attn_workspace(...) bytes */
+CSA2_API size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
+                                  int32_t window);
+CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_t H, int32_t D,
+                               const uint8_t* kv_codes, const uint8_t* kv_scales,
+                               int64_t cap_rows, csa2_seqs_t seqs,
+                               const int32_t* indices, int32_t topk,
+                               const uint16_t* swa_kv, int64_t swa_rows,
+                               const int64_t* swa_start, const int64_t* q_pos,
+                               int32_t window, float softmax_scale,
+                               float* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Status word helpers. */
+/* Enqueue a clear of the status word at the start of `workspace`. */
+CSA2_API csa2_status_t csa2_status_reset(void* workspace, void* stream);
+/* Wait for `stream`, then return the first error any kernel recorded in the status
+ * word of `workspace` since the last reset (CSA2_OK if none). */
+CSA2_API csa2_status_t csa2_status_fetch(const void* workspace, void* stream);
+/* Static text for a status code. */
+CSA2_API const char* csa2_status_string(csa2_status_t status);
+/* Number of streaming multiprocessors of the current device (0 on error). */
+CSA2_API int32_t csa2_device_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

@@ -1,0 +1,102 @@
+"""The C-ABI library loads and exports every entry point of include/csa2.h; host-side
+argument checks return their status codes without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_kv_cache_03_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_lib.build()
+    from fp4_kv_cache_03_b200 import csa2
+    return csa2.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "csa2.h"), encoding="utf-8").read()
+    return sorted(set(re.findall(r"^CSA2_API[^;(]*?\b(csa2_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    from fp4_kv_cache_03_b200 import csa2
+    assert csa2.status_string(0) == "ok"
+    assert "timed out" in csa2.status_string(csa2.ERR_TIMEOUT)
+
+
+def test_workspace_sizes(L):
+    from fp4_kv_cache_03_b200 import csa2
+    assert csa2.quant_append_workspace() == 256
+    a = csa2.index_full_workspace(1, 131072, 512, 0, 8)
+    b = csa2.index_full_workspace(1, 131072, 512, 2048, 8)
+    assert a >= 256 + 131072 * 4 and b > a
+    assert csa2.index_pool_workspace(1, 2048, 8, 512) >= 256 + 16384 * 4
+    assert csa2.sparse_attn_workspace(1, 64, 512, 512, 128) >= 256
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: the checks below return first
+
+
+def test_host_checks_quant_append(L):
+    from fp4_kv_cache_03_b200 import csa2
+    st = L.csa2_quant_append(FAKE, 4, 24, FAKE, FAKE, FAKE, 100, None, None, 0, FAKE, 256, None)
+    assert st == csa2.ERR_INVALID_ARG                        # D not a multiple of 32
+    st = L.csa2_quant_append(FAKE, 4, 64, FAKE, FAKE, FAKE, 100, None, None, 0, FAKE, 16, None)
+    assert st == csa2.ERR_CAPACITY                           # workspace too small
+    st = L.csa2_quant_append(FAKE, 0, 64, FAKE, FAKE, FAKE, 100, None, None, 0, FAKE, 256, None)
+    assert st == csa2.OK                                     # nothing to do
+
+
+def _seqs(n=1, qps=1):
+    from fp4_kv_cache_03_b200 import csa2
+    return csa2.Seqs(n, qps, FAKE, FAKE)
+
+
+def test_host_checks_index(L):
+    from fp4_kv_cache_03_b200 import csa2
+    args = lambda H_I=4, d_I=64, topk=64, ws=1 << 30, pool_blocks=0, block=8: (
+        FAKE, FAKE, 1, H_I, d_I, FAKE, 4096, _seqs(), None, 4096, topk, FAKE, pool_blocks, block,
+        FAKE, ctypes.c_void_p(0x100000), ws, None)
+    assert L.csa2_index_full(*args(H_I=0)) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_index_full(*args(H_I=33)) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_index_full(*args(d_I=96)) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_index_full(*args(topk=0)) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_index_full(*args(pool_blocks=16, block=3)) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_index_full(*args(ws=1024)) == csa2.ERR_CAPACITY
+    a = list(args())
+    a[7] = _seqs(2, 1)                                       # 2 sequences x 1 != num_q
+    assert L.csa2_index_full(*a) == csa2.ERR_INVALID_ARG
+    pa = (FAKE, FAKE, 1, 4, 64, FAKE, 4096, _seqs(), None, FAKE, 16, 4, 64, FAKE,
+          ctypes.c_void_p(0x100000), 1 << 30, None)
+    assert L.csa2_index_pool(*pa) == csa2.ERR_UNSUPPORTED    # block must be 8
+
+
+def test_host_checks_attention(L):
+    from fp4_kv_cache_03_b200 import csa2
+    def call(H=16, D=128, topk=64, window=128, ws=1 << 30):
+        return L.csa2_sparse_attn(FAKE, 1, H, D, FAKE, FAKE, 100, _seqs(), FAKE, topk, FAKE, 100,
+                                  FAKE, FAKE, window, 0.1, FAKE, None,
+                                  ctypes.c_void_p(0x100000), ws, None)
+    assert call(H=12) == csa2.ERR_UNSUPPORTED
+    assert call(D=96) == csa2.ERR_UNSUPPORTED
+    assert call(topk=4096) == csa2.ERR_INVALID_ARG
+    assert call(ws=300) == csa2.ERR_CAPACITY
+
+
+def test_device_query_without_gpu_is_harmless(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.csa2_device_sms() == 0
