@@ -45,6 +45,9 @@ _SIGS = {
     "csa2_index_full": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                   c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p, c_int32,
                                   c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa2_index_full_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                          c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p,
+                                          c_int32, c_int32, c_void_p, c_void_p]),
     "csa2_index_pool_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32]),
     "csa2_index_pool": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                   c_int64, Seqs, c_void_p, c_void_p, c_int32, c_int32, c_int32,
@@ -146,6 +149,20 @@ def index_full(qI, w, idx_k, seqs: Seqs, topk, indices, ws, max_visible, q_visib
                                  seqs, _p(q_visible), int(max_visible), topk, _p(indices),
                                  pool_blocks, block, _p(pool), _p(ws), ws.numel(), _s(stream)),
            "csa2_index_full")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def index_full_noalloc(qI, w, idx_k, seqs: Seqs, topk, indices, max_visible, q_visible=None,
+                       pool_blocks=0, block=8, pool=None, stream=None):
+    """csa2_index_full with the library's own fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory); see include/csa2.h."""
+    num_q, H_I, d_I = qI.shape
+    _check(lib().csa2_index_full_noalloc(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k),
+                                         idx_k.shape[0], seqs, _p(q_visible), int(max_visible),
+                                         topk, _p(indices), pool_blocks, block, _p(pool),
+                                         _s(stream)), "csa2_index_full_noalloc")
 
 
 def index_pool_workspace(num_q, pool_blocks, block, topk) -> int:

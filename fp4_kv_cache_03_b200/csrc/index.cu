@@ -18,6 +18,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -741,4 +742,58 @@ extern "C" csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int
   return run_index<true>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, 0x7FFFFFFF,
                          topk, indices, pool_blocks, block, nullptr, pool, workspace, ws_bytes,
                          (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------------
+// csa2_index_full_noalloc: the same computation with the library's own scratch array,
+// for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------------
+// Scratch of the no-allocation entry point.  Every GPU that loads the library holds it
+// until exit.  In host code this name is only a stand-in for the device array: the kernels
+// get its device address, looked up below with the device current.
+static __device__ __align__(256) unsigned char csa2_index_scratch[CSA2_INDEX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of csa2_index_scratch on the current device (looked up once per device).
+void* index_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, csa2_index_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_addr[dev] = p;
+  }
+  return g_scratch_addr[dev];
+}
+}  // namespace
+
+extern "C" csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float* w,
+                                                 int32_t num_q, int32_t H_I, int32_t d_I,
+                                                 const uint16_t* idx_k, int64_t cap_rows,
+                                                 csa2_seqs_t seqs, const int32_t* q_visible,
+                                                 int32_t max_visible, int32_t topk,
+                                                 int32_t* indices, int32_t pool_blocks,
+                                                 int32_t block, int32_t* pool, void* stream) {
+  if (max_visible < 0) return CSA2_ERR_INVALID_ARG;
+  if (pool_blocks < 0 || pool_blocks > 8192) return CSA2_ERR_UNSUPPORTED;
+  const size_t need = csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks,
+                                                pool_blocks > 0 ? block : 8);
+  if (need == 0 || need > (size_t)CSA2_INDEX_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_CAPACITY;
+  void* ws = index_scratch_address();
+  if (!ws) return CSA2_ERR_CUDA;
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices, ws);
+  if (st != CSA2_OK || num_q == 0) return st;
+  if (pool_blocks > 0 && (!pool || !pow2_le32(block))) return CSA2_ERR_UNSUPPORTED;
+  if (pool_blocks == 0) block = 8;
+  // the status word starts clear on every call (the histograms are cleared by run_index)
+  if (cudaMemsetAsync(ws, 0, CSA2_STATUS_BYTES, (cudaStream_t)stream) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  return run_index<false>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, max_visible,
+                          topk, indices, pool_blocks, block, pool, nullptr, ws,
+                          (size_t)CSA2_INDEX_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
 }

@@ -136,6 +136,35 @@ CSA2_API csa2_status_t csa2_index_full(const uint16_t* qI, const float* w, int32
                               void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa2_index_full without a workspace: for callers that cannot allocate device memory.
+ * (The pages have no counterpart; this is a deployment convenience.)  Some callers run
+ * where cudaMalloc is unavailable or forbidden -- inside a host framework that owns the
+ * allocator, a real-time loop that must not allocate, or code that is not allowed to grow
+ * device memory after start-up -- and so cannot provide csa2_index_full's workspace.
+ * This entry point computes exactly what csa2_index_full computes (same arguments minus
+ * the workspace) using scratch memory that the library holds in a fixed-size device array
+ * of CSA2_INDEX_NOALLOC_SCRATCH_BYTES, present on every GPU that loads the library until
+ * the process exits.  It calls no cudaMalloc / cudaFree and no allocating routine.
+ *   - Size limit: if csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks, block)
+ *     exceeds CSA2_INDEX_NOALLOC_SCRATCH_BYTES the call returns CSA2_ERR_CAPACITY and
+ *     enqueues nothing (8 MiB covers one query over 1,048,576 entries with a pool).
+ *   - Set-up: the first call on a device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array and leaves its contents there;
+ *     each call clears what must start at zero.  Calls that overlap on the GPU (different
+ *     streams, or different host threads) race on the array: serialise them.
+ *   - Device-side value errors are handled as in csa2_index_full (skipped / clamped) but
+ *     cannot be fetched: the status word lives in the library's array. */
+#define CSA2_INDEX_NOALLOC_SCRATCH_BYTES (8u << 20)
+CSA2_API csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float* w, int32_t num_q,
+                                               int32_t H_I, int32_t d_I, const uint16_t* idx_k,
+                                               int64_t cap_rows, csa2_seqs_t seqs,
+                                               const int32_t* q_visible, int32_t max_visible,
+                                               int32_t topk, int32_t* indices,
+                                               int32_t pool_blocks, int32_t block, int32_t* pool,
+                                               void* stream);
+
+/* ---------------------------------------------------------------------------------
  * a5. Reindex over the pool ([SURV] §2.2.2: Reindex reuses main KV and indexer K but has
  * its own indexer Q and re-selects; [MTP] "CSA2：…": Reindex layers only score inside the
  * bounded pool).  Candidates of query q: positions block*pool[q][i] + r, r < block, for
