@@ -1,28 +1,41 @@
-// a7: sparse attention over the selected FP4 entries joined with the layer's own
-// sliding window, one softmax over both sets.
+// a7: sparse attention over the selected FP4 entries joined with the layer's own sliding
+// window, one softmax over both sets.
 // Pages: aprilzz.com "DeepSeek V4.1 Flash 发布…", sections "把 prefill 砍掉一半" (every layer
-// keeps a 128-token window) and "CSA2：在层的维度上共享缓存" (each layer keeps its own main
-// Q and window KV; Reuse layers attend with the latest indices);
-// "FP4 KV 与部署层的几个改动" (E2M1 + per-16-channel E4M3, dequantised for the product).
+// keeps a 128-token window), "CSA2：在层的维度上共享缓存" (each layer keeps its own main Q
+// and window KV; Reuse layers attend with the latest indices) and "FP4 KV 与部署层的几个改动"
+// (E2M1 values with one E4M3 scale per 16 channels).
 //
-// Split over key slots: CTA (split, q) gathers 64 slots of the list
-// [indices[q][0..topk) ; window positions], dequantises FP4 rows in registers to bf16
-// (exact: a 2-bit-mantissa value times a 4-bit-mantissa scale), and computes
-// S = scale * Q K^T, a partial softmax (m, l) and O = P V for all heads; a second kernel
-// merges the splits by log-sum-exp.
+// One CTA handles a range of 128-key tiles of one query.  The key slots of a query are
+// [indices[q][0..topk) ; window positions t-W+1 .. t].  Per tile:
+//   gather   all 8 warps load the tile's rows -- FP4 rows are dequantised in registers to
+//            bf16 (exact: a 2-bit-mantissa code times a 4-bit-mantissa scale), window rows
+//            are copied with cp.async -- into a 128-byte-swizzled [128 keys x D] tile;
+//   S^T      one thread issues tcgen05.mma: S^T[key, head] = KV[key, :] . Q[head, :]
+//            (M = 128 keys, N = heads, K = D; Q arrives once by TMA);
+//   softmax  warps 0-3 read S^T from TMEM (one key per thread), form per-head maxima and
+//            sums with warp reduce-scatters, keep a lazily rescaled running max per head,
+//            and write P (bf16) as [key][head] rows -- an MN-major operand;
+//   O^T      tcgen05.mma: O^T[d, head] += V^T[d, key] . P^T[key, head], reading the same
+//            swizzled KV tile as an MN-major operand (M = 128 dims per slab, N = heads).
+// The last tile's O^T is normalised and written; when a query is split over several CTAs
+// they write (m, l, O) partials that a small kernel merges by log-sum-exp.
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 
 namespace csa2 {
 namespace {
 
-constexpr int kSlots = 64;          // key slots per CTA
-constexpr int kAttnThreads = 256;
+constexpr int kThreads = 256;                // 8 warps
+constexpr int kTile = 128;                   // keys per tile (MMA M)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;         // rescale O only when a max grows by > 2^8
 
 struct AttnArgs {
-  const uint16_t* q;
-  int num_q, H, D;
+  int num_q;
   const uint8_t* codes;
   const uint8_t* scales;
   int64_t cap_rows;
@@ -36,214 +49,450 @@ struct AttnArgs {
   const int64_t* swa_start;
   const int64_t* q_pos;
   int window;
-  float scale;
-  int nsplit;
-  float* part_o;   // [num_q][nsplit][H][D]
-  float* part_ml;  // [num_q][nsplit][H][2]
+  int H;                                     // real heads (<= kN); the rest are padding
+  float scale_log2;                          // softmax_scale * log2(e)
+  int n_tiles;                               // tiles of the slot list
+  int nsplit, tiles_per_split;
+  float* part_o;                             // [num_q][nsplit][H][D]  (nsplit > 1)
+  float* part_ml;                            // [num_q][nsplit][H][2]  log2-domain m, l
   float* out;
   float* lse;
   int* status;
 };
 
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  const uint32_t m = c & 7u;
-  const float mag = m < 4 ? 0.5f * (float)m : (m == 4 ? 2.0f : (m == 5 ? 3.0f : (m == 6 ? 4.0f : 6.0f)));
+constexpr int kN = 64;                       // MMA N: heads, padded to 64
+
+template <int H>
+struct AttnSmem {
+  uint64_t bar_q, bar_s, bar_o;
+  uint32_t tmem_base;
+  int abort;
+  int rescale;
+  float m_ref[H];
+  float l_acc[H];
+  float alpha[H];
+  float red[4][H];
+  int valid[kTile];
+};
+
+// e2m1 code (4 bits) -> value: exponent field e (2 bits, bias 1), mantissa bit m;
+// e = 0 is the subnormal m * 0.5, else (1 + m/2) * 2^(e-1)
+__device__ __forceinline__ float e2m1_val(uint32_t c) {
+  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+  const float mag = e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : 0.5f * (float)m;
   return (c & 8u) ? -mag : mag;
 }
-__device__ __forceinline__ float e4m3_value(uint32_t b) {
+// non-negative e4m3 scale byte -> value (bias 7; exponent field 0 is subnormal m * 2^-9)
+__device__ __forceinline__ float e4m3_val(uint32_t b) {
   const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-  float v = (e == 0) ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  const float v = (e == 0) ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
   return (b & 0x80u) ? -v : v;
 }
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
 
-__global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int split = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
-  const int H = a.H, D = a.D, KD = D + 8;  // padded key rows
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sK = sQ + (size_t)H * D;
-  float* sS = reinterpret_cast<float*>(sK + (size_t)kSlots * KD);   // [H][kSlots]
-  float* sM = sS + (size_t)H * kSlots;                                // [H]
-  int* sValid = reinterpret_cast<int*>(sM + H);                       // [kSlots]
-
-  const int seq = q / a.q_per_seq;
-  const int64_t t = a.q_pos[q];
-  const int64_t w0 = t - a.window + 1 > 0 ? t - a.window + 1 : 0;
-  const int n_win = (int)(t + 1 - w0 < 0 ? 0 : t + 1 - w0);
-
-  // Q -> shared
-  const uint4* gq = reinterpret_cast<const uint4*>(a.q + (int64_t)q * H * D);
-  for (int i = tid; i < H * D / 8; i += kAttnThreads) reinterpret_cast<uint4*>(sQ)[i] = gq[i];
-
-  // gather + dequantise this split's key slots (one 16-channel group per item)
-  const int gpr = D / 16;
-  for (int it = tid; it < kSlots * gpr; it += kAttnThreads) {
-    const int j = it / gpr, g = it % gpr;
-    const int slot = split * kSlots + j;
-    __nv_bfloat16* dst = sK + (size_t)j * KD + g * 16;
-    bool ok = false;
-    if (slot < a.topk) {
-      const int p = a.indices[(int64_t)q * a.topk + slot];
-      if (p >= 0) {
-        const int64_t row = a.seq_start[seq] + p;
-        if (p >= a.seq_len[seq]) {
-          report(a.status, CSA2_ERR_INVALID_ARG);
-        } else if (row >= a.cap_rows) {
-          report(a.status, CSA2_ERR_CAPACITY);
-        } else {
-          const uint2 c = __ldg(reinterpret_cast<const uint2*>(a.codes + row * (D / 2) + g * 8));
-          const float s = e4m3_value(__ldg(a.scales + row * gpr + g));
-          const uint32_t cw[2] = {c.x, c.y};
-          __align__(16) __nv_bfloat16 v[16];
+// Reduce-scatter of v[0..N) across the 32 lanes of a warp (compile-time recursion over the
+// lane bits 16, 8, 4, 2, 1): at each step a lane keeps the half of its values selected by
+// its lane bit and combines it with the other half from its partner.  Afterwards lane l
+// holds the warp-wide result for heads [kOwn*l, kOwn*l + kOwn) in v[0..kOwn), kOwn = N/32.
+template <int N, int BIT, bool kMax>
+__device__ __forceinline__ void reduce_scatter_step(float* v, int lane) {
+  if constexpr (BIT > 0) {
+    static_assert(N >= 2, "needs at least two values per lane");
+    constexpr int half = N / 2;
+    const bool upper = (lane & BIT) != 0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            v[i] = __float2bfloat16_rn(e2m1_value((cw[i >> 3] >> (4 * (i & 7))) & 15u) * s);
-          reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<uint4*>(v)[0];
-          reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<uint4*>(v)[1];
-          ok = true;
-        }
-      } else if (p < -1) {
-        report(a.status, CSA2_ERR_INVALID_ARG);
-      }
-    } else if (slot - a.topk < n_win) {
-      const int64_t row = a.swa_start[seq] + w0 + (slot - a.topk);
-      if (row < 0 || row >= a.swa_rows) {
-        report(a.status, CSA2_ERR_CAPACITY);
-      } else {
-        const uint4* src = reinterpret_cast<const uint4*>(a.swa + row * D + g * 16);
-        reinterpret_cast<uint4*>(dst)[0] = __ldg(src);
-        reinterpret_cast<uint4*>(dst)[1] = __ldg(src + 1);
-        ok = true;
-      }
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[i + half] : v[i];
+      const float send = upper ? v[i] : v[i + half];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, BIT);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
     }
-    if (!ok) {
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(0, 0, 0, 0);
-    }
-    if (g == 0) sValid[j] = ok ? 1 : 0;
+    reduce_scatter_step<half, BIT / 2, kMax>(v, lane);
   }
-  __syncthreads();
+}
 
-  // S[h][j] = scale * Q[h] . K[j]
-  {
-    const int j = tid & (kSlots - 1), hg = tid >> 6;   // 4 head groups
-    float acc[32];
-    const int nh = H / 4;                              // heads per thread (<= 32)
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
+  constexpr int H = kN;
+  constexpr int kChunks = D / 64;            // 64-element (128-byte) column chunks
+  constexpr int kSlabs = D / 128;            // O^T slabs of 128 dims (MMA M)
+  constexpr uint32_t kQChunk = H * 128;      // bytes of one Q chunk ([H rows][128 B])
+  constexpr uint32_t kQBytes = kChunks * kQChunk;
+  constexpr uint32_t kKVChunk = kTile * 128;  // 16 KB
+  constexpr uint32_t kTmemCols = (H + kSlabs * H) <= 32 ? 32 : ((H + kSlabs * H) <= 64 ? 64 : ((H + kSlabs * H) <= 128 ? 128 : ((H + kSlabs * H) <= 256 ? 256 : 512)));
+  static_assert(D % 128 == 0 && D <= 512, "shape");
+  const int Hr = a.H;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ AttnSmem<H> ss;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sKV = sQ + ((kQBytes + 1023) / 1024) * 1024;
+  uint8_t* sP = sKV + kChunks * kKVChunk;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, q = blockIdx.y;
+  const int seq = q / a.q_per_seq;
+  const int t_begin = split * a.tiles_per_split;
+  const int t_end = min(a.n_tiles, t_begin + a.tiles_per_split);
+  volatile int* abort = &ss.abort;
+
+  if (tid == 0) {
+    mbar_init(&ss.bar_q, 1);
+    mbar_init(&ss.bar_s, 1);
+    mbar_init(&ss.bar_o, 1);
+    ss.abort = 0;
+    fence_barrier_init();
+  }
+  if (tid < H) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
+  if (Hr < H) {  // rows of padding heads must read as zero; TMA writes rows < Hr only
+    for (uint32_t i = tid * 16; i < kQBytes; i += kThreads * 16)
+      *reinterpret_cast<uint4*>(sQ + i) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) { tmem_alloc(&ss.tmem_base, kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss.tmem_base;
+  const uint32_t tS = tmem;                  // S^T: columns [0, H)
+  const uint32_t tO = tmem + H;              // O^T slab j: columns [H + jH, H + (j+1)H)
+
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * Hr * 128);
+    for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunk, &tm_q, c * 64, q * Hr, &ss.bar_q);
+  }
+
+  const int64_t row0 = a.seq_start[seq];
+  const int slen = a.seq_len[seq];
+  const int64_t t_q = a.q_pos[q];
+  const int64_t w0 = t_q - a.window + 1 > 0 ? t_q - a.window + 1 : 0;
+  const int n_win = (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0);
+  const int64_t wrow0 = a.swa_start[seq] + w0;
+
+  const uint32_t idesc_s = idesc_bf16(kTile, H);
+  const uint32_t idesc_o = idesc_bf16(kTile, H, true, true);
+  uint32_t ph_s = 0, ph_o = 0;
+  bool q_ready = false, o_init = false, o_pending = false;
+
+  for (int t = t_begin; t < t_end && !*abort; ++t) {
+    // the previous tile's O^T MMA must be done before its KV / P buffers are rewritten
+    if (o_pending) {
+      if (!mbar_wait(&ss.bar_o, ph_o, abort, a.status)) break;
+      ph_o ^= 1;
+      o_pending = false;
+      tc_fence_after();
+    }
+    // ------------------------------ gather ------------------------------
+    constexpr int kParts = D / 32;                 // 32-column parts per row
+    constexpr int kRowsPerIter = kThreads / kParts;
+    const int part = tid % kParts;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-    const __nv_bfloat16* kr = sK + (size_t)j * KD;
-    for (int d = 0; d < D; d += 8) {
-      const uint4 kv = *reinterpret_cast<const uint4*>(kr + d);
-      const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kv);
-      float kf[8];
+    for (int r0 = 0; r0 < kTile; r0 += kRowsPerIter) {
+      const int r = r0 + tid / kParts;
+      const int slot = t * kTile + r;
+      uint8_t* row_smem = sKV + r * 128;
+      int kind = 0;                                // 0 invalid, 1 fp4 row, 2 window row
+      int64_t grow = 0;
+      if (slot < a.topk) {
+        const int p = a.indices[(int64_t)q * a.topk + slot];
+        if (p >= 0 && p < slen) {
+          grow = row0 + p;
+          if (grow < a.cap_rows) kind = 1; else report(a.status, CSA2_ERR_CAPACITY);
+        } else if (p != -1) {
+          report(a.status, CSA2_ERR_INVALID_ARG);
+        }
+      } else if (slot - a.topk < n_win) {
+        grow = wrow0 + (slot - a.topk);
+        if (grow >= 0 && grow < a.swa_rows) kind = 2; else report(a.status, CSA2_ERR_CAPACITY);
+      }
+      if (part == 0) ss.valid[r] = kind != 0;
+      // this part covers columns [32*part, 32*part + 32): 4 units of 8 bf16
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(k2[i]);
-        kf[2 * i] = f.x; kf[2 * i + 1] = f.y;
+        const int u = 4 * part + i;                // 16-byte unit of the row
+        uint8_t* dst = row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4);
+        if (kind == 2) {
+          cp_async16(dst, a.swa + grow * D + u * 8);
+        } else if (kind == 0) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
       }
+      if (kind == 1) {
+        const uint4 c = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
+        const uint16_t sc2 = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
+        const float s0 = e4m3_val(sc2 & 0xFFu), s1 = e4m3_val(sc2 >> 8);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (i < nh) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(sQ + (size_t)(hg + 4 * i) * D + d);
-          const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
+        for (int i = 0; i < 4; ++i) {              // unit i: codes of cw[i] (8 values)
+          const float s = i < 2 ? s0 : s1;
+          uint4 o;
+          uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 f = __bfloat1622float2(q2[u]);
-            acc[i] = fmaf(f.x, kf[2 * u], acc[i]);
-            acc[i] = fmaf(f.y, kf[2 * u + 1], acc[i]);
+          for (int k = 0; k < 4; ++k)
+            ow[k] = pack_bf16(e2m1_val((cw[i] >> (8 * k)) & 15u) * s,
+                              e2m1_val((cw[i] >> (8 * k + 4)) & 15u) * s);
+          const int u = 4 * part + i;
+          *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
+        }
+      }
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    const int any = __syncthreads_or(ss.valid[tid & (kTile - 1)]);
+    if (!any) continue;
+
+    // ------------------------------ S^T = KV . Q^T ------------------------------
+    if (tid == 0) {
+      bool ok = true;
+      if (!q_ready) { ok = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = ok; }
+      if (ok) {
+        tc_fence_after();
+        const uint32_t kv = smem_u32(sKV), qs = smem_u32(sQ);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(kv + (k >> 2) * kKVChunk + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(qs + (k >> 2) * kQChunk + (k & 3) * 32, 16, 1024);
+          umma_bf16(tS, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&ss.bar_s);
+      }
+    }
+
+    // ------------------------------ softmax (warps 0-3) ------------------------------
+    if (warp < 4) {
+      const int r = warp * 32 + lane;             // key row = TMEM lane
+      if (tid == 0) ss.rescale = 0;
+      float v[H];
+      bool ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < H; c += 16) tmem_ld16(tS + ((uint32_t)(warp * 32) << 16) + c, v + c);
+        const bool valid = ss.valid[r] != 0;
+#pragma unroll
+        for (int h = 0; h < H; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
+        // per-head tile maximum
+        float red[H];
+#pragma unroll
+        for (int h = 0; h < H; ++h) red[h] = v[h];
+        reduce_scatter_step<H, 16, true>(red, lane);
+        constexpr int kOwn = H / 32;
+#pragma unroll
+        for (int i = 0; i < kOwn; ++i) ss.red[warp][kOwn * lane + i] = red[i];
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (ok) {
+        if (tid < H) {
+          const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
+          ss.alpha[tid] = mt;                     // stash the tile max
+          if (mt > ss.m_ref[tid] + kRescaleLog2) ss.rescale = 1;
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int need = ss.rescale;
+      if (ok && need) {
+        // move every head's reference max up to its running max; O and l scale by alpha
+        if (tid < H) {
+          const float mo = ss.m_ref[tid];
+          const float mn = fmaxf(mo, ss.alpha[tid]);
+          const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+          ss.alpha[tid] = al;
+          ss.l_acc[tid] *= al;
+          ss.m_ref[tid] = mn;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (o_init) {
+#pragma unroll
+          for (int j = 0; j < kSlabs; ++j) {
+#pragma unroll
+            for (int c = 0; c < H; c += 16) {
+              float o[16];
+              const uint32_t ta = tO + ((uint32_t)(warp * 32) << 16) + j * H + c;
+              tmem_ld16(ta, o);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] *= ss.alpha[c + i];
+              tmem_st16(ta, o);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      if (ok) {
+        // p = 2^(s - m_ref), rounded to bf16; P row r = [heads] (MN-major operand)
+        float psum[H];
+#pragma unroll
+        for (int u = 0; u < H / 8; ++u) {
+          uint4 pk;
+          uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int h = 8 * u + 2 * k;
+            const float p0 = exp2f(v[h] - ss.m_ref[h]);
+            const float p1 = exp2f(v[h + 1] - ss.m_ref[h + 1]);
+            pw[k] = pack_bf16(p0, p1);
+            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&pw[k]);
+            const float2 f = __bfloat1622float2(b);
+            psum[h] = f.x;
+            psum[h + 1] = f.y;
+          }
+          *reinterpret_cast<uint4*>(sP + r * 128 + ((u ^ (r & 7)) << 4)) = pk;
+        }
+        reduce_scatter_step<H, 16, false>(psum, lane);
+        constexpr int kOwn = H / 32;
+#pragma unroll
+        for (int i = 0; i < kOwn; ++i) ss.red[warp][kOwn * lane + i] = psum[i];
+        fence_proxy_async_smem();
+        tc_fence_before();
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (ok) {
+        if (tid < H) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
+        // ------------------------------ O^T += V^T . P^T ------------------------------
+        if (tid == 0) {
+          tc_fence_after();
+          const uint32_t kv = smem_u32(sKV), ps = smem_u32(sP);
+#pragma unroll
+          for (int j = 0; j < kSlabs; ++j) {
+#pragma unroll
+            for (int k = 0; k < kTile / 16; ++k) {
+              const uint64_t ad = sdesc_sw128(kv + (2 * j) * kKVChunk + k * 2048, kKVChunk, 1024);
+              const uint64_t bd = sdesc_sw128(ps + k * 2048, 8192, 1024);
+              umma_bf16(tO + j * H, ad, bd, idesc_o, (o_init || k > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&ss.bar_o);
+        }
+      }
+      ph_s ^= 1;
+    }
+    __syncthreads();
+    o_init = true;
+    o_pending = true;
+  }
+
+  // ------------------------------ epilogue ------------------------------
+  if (o_pending) {
+    if (mbar_wait(&ss.bar_o, ph_o, abort, a.status)) tc_fence_after();
+  }
+  __syncthreads();
+  if (warp < 4 && !*abort) {
+    const bool partial = a.nsplit > 1;
+    float* dst = partial ? a.part_o + (((int64_t)q * a.nsplit + split) * Hr) * D
+                         : a.out + (int64_t)q * Hr * D;
+#pragma unroll
+    for (int j = 0; j < kSlabs; ++j) {
+      const int d = j * 128 + warp * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < H; c += 16) {
+        float o[16];
+        if (o_init) tmem_ld16(tO + ((uint32_t)(warp * 32) << 16) + j * H + c, o);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (c + i < Hr) {
+            const float l = ss.l_acc[c + i];
+            float val = o_init ? o[i] : 0.0f;
+            if (!partial) val = (l > 0.0f) ? val / l : 0.0f;
+            dst[(int64_t)(c + i) * D + d] = val;
           }
         }
       }
     }
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i < nh) sS[(size_t)(hg + 4 * i) * kSlots + j] = sValid[j] ? acc[i] * a.scale : -INFINITY;
-  }
-  __syncthreads();
-
-  // partial softmax per head: p = exp(s - m), m = max, l = sum p
-  float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * H) * 2;
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int h = warp; h < H; h += kAttnThreads / 32) {
-      float* row = sS + (size_t)h * kSlots;
-      const float x0 = row[lane], x1 = row[lane + 32];
-      float m = fmaxf(x0, x1);
-      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float p0 = (x0 == -INFINITY) ? 0.0f : expf(x0 - m);
-      const float p1 = (x1 == -INFINITY) ? 0.0f : expf(x1 - m);
-      row[lane] = p0;
-      row[lane + 32] = p1;
-      float l = p0 + p1;
-      for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      if (lane == 0) { ml[2 * h] = m; ml[2 * h + 1] = l; }
-    }
-  }
-  __syncthreads();
-
-  // O[h][d] = sum_j p[h][j] K[j][d]  (two dims, 16 heads per pass)
-  {
-    const int half = D / 2;
-    const int dp = tid % half, hgrp = tid / half, hstep = (kAttnThreads / half) * 16;
-    float* po = a.part_o + (((int64_t)q * a.nsplit + split) * H) * D;
-    for (int h0 = hgrp * 16; h0 < H; h0 += hstep) {
-      float acc0[16], acc1[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) { acc0[i] = 0.0f; acc1[i] = 0.0f; }
-      for (int j = 0; j < kSlots; ++j) {
-        const float2 kv =
-            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sK + (size_t)j * KD + 2 * dp));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p = sS[(size_t)(h0 + i) * kSlots + j];
-          acc0[i] = fmaf(p, kv.x, acc0[i]);
-          acc1[i] = fmaf(p, kv.y, acc1[i]);
-        }
+    if (tid < Hr) {
+      const float m = ss.m_ref[tid], l = ss.l_acc[tid];
+      if (partial) {
+        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + tid) * 2;
+        ml[0] = (l > 0.0f) ? m : -INFINITY;
+        ml[1] = l;
+      } else if (a.lse) {
+        a.lse[(int64_t)q * Hr + tid] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        *reinterpret_cast<float2*>(po + (size_t)(h0 + i) * D + 2 * dp) = make_float2(acc0[i], acc1[i]);
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads) attn_merge_kernel(const AttnArgs a) {
-  const int q = blockIdx.x;
-  const int H = a.H, D = a.D;
-  for (int h = 0; h < H; ++h) {
-    const float* ml = a.part_ml + ((int64_t)q * a.nsplit * H + h) * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, ml[(int64_t)s * H * 2]);
-    float L = 0.0f;
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float m = ml[(int64_t)s * H * 2];
-      if (m != -INFINITY) L += expf(m - M) * ml[(int64_t)s * H * 2 + 1];
-    }
-    float* o = a.out + ((int64_t)q * H + h) * D;
-    for (int d = threadIdx.x; d < D; d += kAttnThreads) {
-      float acc = 0.0f;
-      for (int s = 0; s < a.nsplit; ++s) {
-        const float m = ml[(int64_t)s * H * 2];
-        if (m != -INFINITY)
-          acc += expf(m - M) * a.part_o[(((int64_t)q * a.nsplit + s) * H + h) * D + d];
-      }
-      o[d] = L > 0.0f ? acc / L : 0.0f;
-    }
-    if (a.lse && threadIdx.x == 0) a.lse[(int64_t)q * H + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+// merge the split partials of one (query, head): weights 2^(m_s - M)
+template <int D>
+__global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a, int H) {
+  const int q = blockIdx.x, h = blockIdx.y;
+  const int ns = a.nsplit;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.part_ml[(((int64_t)q * ns + s) * H + h) * 2]);
+  float L = 0.0f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int d = threadIdx.x * 4;
+  for (int s = 0; s < ns; ++s) {
+    const float* ml = a.part_ml + (((int64_t)q * ns + s) * H + h) * 2;
+    if (ml[0] == -INFINITY) continue;
+    const float wgt = exp2f(ml[0] - M);
+    L += wgt * ml[1];
+    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (((int64_t)q * ns + s) * H + h) * D + d);
+    acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
   }
+  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+  *reinterpret_cast<float4*>(a.out + ((int64_t)q * H + h) * D + d) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (a.lse && threadIdx.x == 0)
+    a.lse[(int64_t)q * H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
-size_t attn_smem(int H, int D) {
-  return (size_t)H * D * 2 + (size_t)kSlots * (D + 8) * 2 + (size_t)H * kSlots * 4 + H * 4 +
-         kSlots * 4;
+// ---------------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------------
+inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int n_tiles_of(int topk, int window) { return (topk + window + kTile - 1) / kTile; }
+
+int nsplit_of(int num_q, int n_tiles) {
+  if (n_tiles <= 1) return 1;
+  return std::max(1, std::min(n_tiles, 512 / std::max(1, num_q)));
+}
+
+size_t attn_smem_bytes(int D) {
+  const size_t q = ((size_t)(D / 64) * kN * 128 + 1023) / 1024 * 1024;
+  return 1024 + q + (size_t)(D / 64) * kTile * 128 + kTile * 128;
 }
 
 bool attn_shape_ok(int H, int D) {
-  const bool d_ok = D == 32 || D == 64 || D == 128 || D == 256 || D == 512;
-  return d_ok && H >= 16 && H <= 128 && (H % 16) == 0 && attn_smem(H, D) <= 200 * 1024;
+  return H >= 1 && H <= kN && (D == 128 || D == 256 || D == 512);
 }
 
-inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <int D>
+cudaError_t launch(const AttnArgs& a, const CUtensorMap& tm, cudaStream_t st) {
+  const size_t smem = attn_smem_bytes(D);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<D><<<dim3(a.nsplit, a.num_q), kThreads, smem, st>>>(tm, a);
+  if (a.nsplit > 1) attn_merge_kernel<D><<<dim3(a.num_q, a.H), D / 4, 0, st>>>(a, a.H);
+  return cudaGetLastError();
+}
 
 }  // namespace
 }  // namespace csa2
@@ -253,10 +502,12 @@ using namespace csa2;
 extern "C" size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
                                              int32_t window) {
   if (num_q < 0 || H < 1 || D < 1 || topk < 0 || window < 0) return 0;
-  const int64_t nsplit = ((int64_t)topk + window + kSlots - 1) / kSlots;
+  const int ns = nsplit_of(num_q, n_tiles_of(topk, window));
   size_t off = CSA2_STATUS_BYTES;
-  off = a256(off + (size_t)num_q * nsplit * H * D * 4);
-  off = a256(off + (size_t)num_q * nsplit * H * 2 * 4);
+  if (ns > 1) {
+    off = a256(off + (size_t)num_q * ns * H * D * 4);
+    off = a256(off + (size_t)num_q * ns * H * 2 * 4);
+  }
   return off;
 }
 
@@ -276,20 +527,26 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   if (!workspace || ws_bytes < csa2_sparse_attn_workspace(num_q, H, D, topk, window))
     return CSA2_ERR_CAPACITY;
   if (num_q == 0) return CSA2_OK;
+  if ((int64_t)num_q * H > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;
   if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
   if (topk > 0 && (!indices || !kv_codes || !kv_scales || cap_rows <= 0)) return CSA2_ERR_INVALID_ARG;
   if (window > 0 && (!swa_kv || !swa_start || swa_rows < 0)) return CSA2_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 7) ||
-      (reinterpret_cast<uintptr_t>(swa_kv) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 15) ||
+      (reinterpret_cast<uintptr_t>(kv_scales) & 1) || (reinterpret_cast<uintptr_t>(swa_kv) & 15) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(out) & 15))
     return CSA2_ERR_INVALID_ARG;
   AttnArgs a{};
-  a.q = q; a.num_q = num_q; a.H = H; a.D = D;
+  a.num_q = num_q;
   a.codes = kv_codes; a.scales = kv_scales; a.cap_rows = cap_rows;
   a.seq_start = seqs.seq_start; a.seq_len = seqs.seq_len; a.q_per_seq = seqs.q_per_seq;
   a.indices = indices; a.topk = topk;
   a.swa = swa_kv; a.swa_rows = swa_rows; a.swa_start = swa_start; a.q_pos = q_pos;
-  a.window = window; a.scale = softmax_scale;
-  a.nsplit = (topk + window + kSlots - 1) / kSlots;
+  a.window = window;
+  a.H = H;
+  a.scale_log2 = softmax_scale * kLog2e;
+  a.n_tiles = n_tiles_of(topk, window);
+  a.nsplit = nsplit_of(num_q, a.n_tiles);
+  a.tiles_per_split = (a.n_tiles + a.nsplit - 1) / a.nsplit;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
   size_t off = CSA2_STATUS_BYTES;
@@ -297,14 +554,22 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   off = a256(off + (size_t)num_q * a.nsplit * H * D * 4);
   a.part_ml = reinterpret_cast<float*>(ws + off);
   a.out = out; a.lse = lse;
+
+  auto fn = attn_encode_fn();
+  if (!fn) return CSA2_ERR_CUDA;
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_q * H};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)H};
+  cuuint32_t estr[2] = {1u, 1u};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), dims, strides, box,
+         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return CSA2_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  if (a.nsplit > 0) {
-    const size_t smem = attn_smem(H, D);
-    if (cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return CSA2_ERR_CUDA;
-    attn_split_kernel<<<dim3(a.nsplit, num_q), kAttnThreads, smem, st>>>(a);
-  }
-  attn_merge_kernel<<<num_q, kAttnThreads, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
+  if (D == 128) e = launch<128>(a, tm, st);
+  else if (D == 256) e = launch<256>(a, tm, st);
+  else e = launch<512>(a, tm, st);
+  return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

@@ -197,8 +197,8 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   l_j = softmax_scale * q[q][h] . row_j;  out[q][h] = sum_j softmax(l)_j row_j;
  *   lse[q][h] = log(sum_j exp(l_j)) (natural log); no rows at all gives out = 0,
  *   lse = -inf.  The two sets share one softmax; a row in both counts twice.
- *   q         device bf16 [num_q][H][D]        H a multiple of 16 in 16..128, D a power of
- *             two in 32..512 (other shapes return CSA2_ERR_UNSUPPORTED)
+ *   q         device bf16 [num_q][H][D]        1 <= H <= 64, D in {128, 256, 512} (other
+ *             shapes return CSA2_ERR_UNSUPPORTED); base 16-byte aligned
  *   indices   device int32 [num_q][topk]       0 <= topk <= 2048
  *   swa_kv    device bf16 [swa_rows][D];  swa_start device int64 [num_seqs] (may be
  *             negative: only rows of window positions are read)

@@ -89,8 +89,10 @@ def test_host_checks_attention(L):
         return L.csa2_sparse_attn(FAKE, 1, H, D, FAKE, FAKE, 100, _seqs(), FAKE, topk, FAKE, 100,
                                   FAKE, FAKE, window, 0.1, FAKE, None,
                                   ctypes.c_void_p(0x100000), ws, None)
-    assert call(H=12) == csa2.ERR_UNSUPPORTED
+    assert call(H=65) == csa2.ERR_UNSUPPORTED
+    assert call(H=0) == csa2.ERR_UNSUPPORTED
     assert call(D=96) == csa2.ERR_UNSUPPORTED
+    assert call(D=64) == csa2.ERR_UNSUPPORTED
     assert call(topk=4096) == csa2.ERR_INVALID_ARG
     assert call(ws=300) == csa2.ERR_CAPACITY
 
