@@ -331,7 +331,9 @@ def run_ours(args, rank, world, local_rank):
     achieved = alg_bytes / full_s / 1e9
     steps_total = args.steps * world
     value = steps_total * n_layers / t_total
-    launches_per_step = (1 if W.append else 0) + 6 * n_index + 2 * n_layers
+    # append 1; each index call: score + select (+ a memset, not a kernel); each
+    # attention: the split kernel, + the merge kernel when split (batch 1 always splits)
+    launches_per_step = (1 if W.append else 0) + 2 * n_index + 2 * n_layers
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,

@@ -73,6 +73,7 @@ struct AttnSmem {
   float alpha[H];
   float red[4][H];
   int valid[kTile];
+  uint32_t lut[256];   // code byte -> (e2m1(low nibble), e2m1(high nibble)) as bf16x2
 };
 
 // e2m1 code (4 bits) -> value: exponent field e (2 bits, bias 1), mantissa bit m;
@@ -91,6 +92,18 @@ __device__ __forceinline__ float e4m3_val(uint32_t b) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+// bf16x2 product; exact here: an e2m1 value times an e4m3 scale has at most 6 significant
+// bits and lies in [2^-10, 2688], so it is representable in bf16
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ float fast_exp2(float x) {   // 2^x (MUFU); 2^-inf = 0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Reduce-scatter of v[0..N) across the 32 lanes of a warp (compile-time recursion over the
@@ -150,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (tid < H) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
+  ss.lut[tid] = pack_bf16(e2m1_val(tid & 15u), e2m1_val((uint32_t)tid >> 4));
   if (Hr < H) {  // rows of padding heads must read as zero; TMA writes rows < Hr only
     for (uint32_t i = tid * 16; i < kQBytes; i += kThreads * 16)
       *reinterpret_cast<uint4*>(sQ + i) = make_uint4(0, 0, 0, 0);
@@ -190,56 +204,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
     // ------------------------------ gather ------------------------------
+    // Three phases so that every global load of the tile is in flight at once: the slot
+    // indices, then the rows (FP4 codes + scales into registers, window rows by cp.async
+    // straight to shared memory), then dequantisation and the swizzled shared stores.
     constexpr int kParts = D / 32;                 // 32-column parts per row
     constexpr int kRowsPerIter = kThreads / kParts;
+    constexpr int kIters = kTile / kRowsPerIter;
     const int part = tid % kParts;
+    const int rsub = tid / kParts;
+    int kind[kIters];                              // 0 invalid, 1 FP4 row, 2 window row
+    int64_t grow[kIters];
 #pragma unroll
-    for (int r0 = 0; r0 < kTile; r0 += kRowsPerIter) {
-      const int r = r0 + tid / kParts;
-      const int slot = t * kTile + r;
-      uint8_t* row_smem = sKV + r * 128;
-      int kind = 0;                                // 0 invalid, 1 fp4 row, 2 window row
-      int64_t grow = 0;
+    for (int it = 0; it < kIters; ++it) {
+      const int slot = t * kTile + it * kRowsPerIter + rsub;
+      kind[it] = 0;
+      grow[it] = 0;
       if (slot < a.topk) {
-        const int p = a.indices[(int64_t)q * a.topk + slot];
-        if (p >= 0 && p < slen) {
-          grow = row0 + p;
-          if (grow < a.cap_rows) kind = 1; else report(a.status, CSA2_ERR_CAPACITY);
-        } else if (p != -1) {
-          report(a.status, CSA2_ERR_INVALID_ARG);
-        }
+        const int p = __ldg(a.indices + (int64_t)q * a.topk + slot);
+        grow[it] = p;                              // resolved below, after all loads issue
+        kind[it] = 1;
       } else if (slot - a.topk < n_win) {
-        grow = wrow0 + (slot - a.topk);
-        if (grow >= 0 && grow < a.swa_rows) kind = 2; else report(a.status, CSA2_ERR_CAPACITY);
+        grow[it] = wrow0 + (slot - a.topk);
+        kind[it] = 2;
       }
-      if (part == 0) ss.valid[r] = kind != 0;
-      // this part covers columns [32*part, 32*part + 32): 4 units of 8 bf16
+    }
+    uint4 cw[kIters];
+    uint32_t sc[kIters];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int u = 4 * part + i;                // 16-byte unit of the row
-        uint8_t* dst = row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4);
-        if (kind == 2) {
-          cp_async16(dst, a.swa + grow * D + u * 8);
-        } else if (kind == 0) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    for (int it = 0; it < kIters; ++it) {
+      const int r = it * kRowsPerIter + rsub;
+      uint8_t* row_smem = sKV + r * 128;
+      if (kind[it] == 1) {
+        const int p = (int)grow[it];
+        if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
+          grow[it] = row0 + p;
+          cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow[it] * (D / 2) + part * 16));
+          sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow[it] * (D / 16) + part * 2));
+        } else {
+          if (p >= slen || p < -1) report(a.status, CSA2_ERR_INVALID_ARG);
+          else if (p >= 0) report(a.status, CSA2_ERR_CAPACITY);
+          kind[it] = 0;
+        }
+      } else if (kind[it] == 2) {
+        if (grow[it] >= 0 && grow[it] < a.swa_rows) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int u = 4 * part + i;
+            cp_async16(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4),
+                       a.swa + grow[it] * D + u * 8);
+          }
+        } else {
+          report(a.status, CSA2_ERR_CAPACITY);
+          kind[it] = 0;
         }
       }
-      if (kind == 1) {
-        const uint4 c = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
-        const uint16_t sc2 = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
-        const float s0 = e4m3_val(sc2 & 0xFFu), s1 = e4m3_val(sc2 >> 8);
-        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {              // unit i: codes of cw[i] (8 values)
-          const float s = i < 2 ? s0 : s1;
+    for (int it = 0; it < kIters; ++it) {
+      const int r = it * kRowsPerIter + rsub;
+      uint8_t* row_smem = sKV + r * 128;
+      if (part == 0) ss.valid[r] = kind[it] != 0;
+      if (kind[it] == 1) {
+        const float s0 = e4m3_val(sc[it] & 0xFFu), s1 = e4m3_val((sc[it] >> 8) & 0xFFu);
+        const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
+        const uint32_t w4[4] = {cw[it].x, cw[it].y, cw[it].z, cw[it].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {              // unit i: 8 values of word w4[i]
+          const uint32_t s2 = i < 2 ? s02 : s12;
           uint4 o;
           uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ow[k] = pack_bf16(e2m1_val((cw[i] >> (8 * k)) & 15u) * s,
-                              e2m1_val((cw[i] >> (8 * k + 4)) & 15u) * s);
+          for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ss.lut[(w4[i] >> (8 * k)) & 0xFFu], s2);
           const int u = 4 * part + i;
           *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
+        }
+      } else if (kind[it] == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int u = 4 * part + i;
+          *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) =
+              make_uint4(0, 0, 0, 0);
         }
       }
     }
@@ -255,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         const uint32_t kv = smem_u32(sKV), qs = smem_u32(sQ);
-#pragma unroll
+#pragma unroll 4
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t ad = sdesc_sw128(kv + (k >> 2) * kKVChunk + (k & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(qs + (k >> 2) * kQChunk + (k & 3) * 32, 16, 1024);
@@ -335,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int h = 8 * u + 2 * k;
-            const float p0 = exp2f(v[h] - ss.m_ref[h]);
-            const float p1 = exp2f(v[h + 1] - ss.m_ref[h + 1]);
+            const float p0 = fast_exp2(v[h] - ss.m_ref[h]);
+            const float p1 = fast_exp2(v[h + 1] - ss.m_ref[h + 1]);
             pw[k] = pack_bf16(p0, p1);
             const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&pw[k]);
             const float2 f = __bfloat1622float2(b);
@@ -359,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) {
           tc_fence_after();
           const uint32_t kv = smem_u32(sKV), ps = smem_u32(sP);
-#pragma unroll
+#pragma unroll 1
           for (int j = 0; j < kSlabs; ++j) {
-#pragma unroll
+#pragma unroll 4
             for (int k = 0; k < kTile / 16; ++k) {
               const uint64_t ad = sdesc_sw128(kv + (2 * j) * kKVChunk + k * 2048, kKVChunk, 1024);
               const uint64_t bd = sdesc_sw128(ps + k * 2048, 8192, 1024);
@@ -383,14 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (mbar_wait(&ss.bar_o, ph_o, abort, a.status)) tc_fence_after();
   }
   __syncthreads();
+  // The KV tile is free once the last O^T MMA has completed: stage O (normalised unless
+  // partial) there as [head][D] fp32, then copy it out with 16-byte stores.
+  const bool partial = a.nsplit > 1;
+  float* so = reinterpret_cast<float*>(sKV);        // [Hr][D] (Hr * D * 4 <= 128 KB)
   if (warp < 4 && !*abort) {
-    const bool partial = a.nsplit > 1;
-    float* dst = partial ? a.part_o + (((int64_t)q * a.nsplit + split) * Hr) * D
-                         : a.out + (int64_t)q * Hr * D;
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < kSlabs; ++j) {
       const int d = j * 128 + warp * 32 + lane;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < H; c += 16) {
         float o[16];
         if (o_init) tmem_ld16(tO + ((uint32_t)(warp * 32) << 16) + j * H + c, o);
@@ -400,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float l = ss.l_acc[c + i];
             float val = o_init ? o[i] : 0.0f;
             if (!partial) val = (l > 0.0f) ? val / l : 0.0f;
-            dst[(int64_t)(c + i) * D + d] = val;
+            so[(c + i) * D + d] = val;
           }
         }
       }
@@ -415,6 +460,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.lse[(int64_t)q * Hr + tid] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
     }
+  }
+  __syncthreads();
+  if (!*abort) {
+    float4* dst4 = reinterpret_cast<float4*>(partial ? a.part_o + (((int64_t)q * a.nsplit + split) * Hr) * D
+                                                     : a.out + (int64_t)q * Hr * D);
+    const float4* src4 = reinterpret_cast<const float4*>(so);
+    const int n4 = Hr * D / 4;
+#pragma unroll 4
+    for (int i = tid; i < n4; i += kThreads) dst4[i] = src4[i];
   }
   tc_fence_before();
   __syncthreads();

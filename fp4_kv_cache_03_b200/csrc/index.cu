@@ -7,14 +7,19 @@
 // (Full/Reindex/Reuse, Top-512, pool of <= 2048 blocks x 8); gkm0120.cn "技术调研报告"
 // §2.2.2 (modes table) and §2.2.3 (hierarchical sparse indexer).
 //
-// Score kernel: persistent, warp-specialised.  Warp 0 streams 128-entry tiles of the
-// bf16 indexer K with TMA (128-byte swizzle) into a ring of shared-memory stages, warp 1
-// issues tcgen05.mma (M = 128 entries, N = padded indexer heads, K = d_I) into a
-// double-buffered TMEM accumulator, warps 2-5 read it back (tcgen05.ld), apply
-// ReLU * w, sum the heads, and write one 32-bit ordered key per entry (plus the block
-// maximum for the pool).  Selection: exact multi-CTA radix select over the keys
-// (11/11/10-bit digits, per-row histograms), then an order-preserving compaction that
-// breaks ties by lowest position.
+// Score kernel: persistent, warp-specialised; each CTA takes one contiguous, equal share
+// of the active 128-entry tiles of all queries (exact balance for ragged batches and
+// causal chunks).  Warp 0 streams tiles of the bf16 indexer K with TMA (128-byte swizzle)
+// into a ring of shared-memory stages, warp 1 issues tcgen05.mma (M = 128 entries,
+// N = indexer heads padded to 16/32, K = d_I) into a double-buffered TMEM accumulator,
+// warps 2-5 read it back (tcgen05.ld), apply ReLU * w, sum the heads and write one 32-bit
+// order-preserving key per entry (plus the block maximum for the pool).  The epilogue also
+// builds the first radix digit's histogram of every row (bits 31..21 of the key).
+// Select kernel: a CTA per 8192-key chunk reads its row's histogram, finds the bin holding
+// the K-th key, and appends the chunk's candidates (keys in that bin or above) to a
+// per-row list in position order; the last CTA of the row (counted with an atomic, no
+// waiting) finishes an exact radix select over the candidates (bits 20..10, then 9..0)
+// and writes the Top-K in ascending position order, lowest position first among ties.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -25,12 +30,13 @@
 namespace csa2 {
 namespace {
 
-constexpr int kTileRows = 128;       // entries per MMA tile (M)
-constexpr int kScoreThreads = 192;   // 6 warps
+constexpr int kTileRows = 128;         // entries per MMA tile (M)
+constexpr int kScoreThreads = 192;     // 6 warps
 constexpr int kSelThreads = 256;
-constexpr int kSelChunk = 8192;      // keys per select CTA
-constexpr int kHistBins = 2048;
-constexpr int kPasses = 3;           // digits: bits 31..21, 20..10, 9..0
+constexpr int kSelChunk = 8192;        // keys per select CTA
+constexpr int kHistBins = 2048;        // first digit: key bits 31..21
+constexpr int kMaxRowsPerLaunch = 4096;
+constexpr int kMaxListChunks = 1024;   // rows longer than this many chunks stream their keys
 
 // ---------------------------------------------------------------------------------
 // visibility
@@ -54,24 +60,34 @@ __device__ __forceinline__ int visible_of(const Seqs& s, int q) {
   return v;
 }
 
+// leading pool entries >= 0 (a pool lists ascending block ids, then -1 padding)
+__device__ __forceinline__ int pool_valid(const int32_t* pool_row, int n) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (pool_row[mid] >= 0) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // ---------------------------------------------------------------------------------
 // score kernel
 // ---------------------------------------------------------------------------------
 struct ScoreArgs {
   Seqs seqs;
   const float* w;
-  int num_q, H_I, d_I, n_pad;      // n_pad: MMA N (multiple of 16)
-  int tiles_per_q;                 // host bound on tiles of one query
+  int q0, num_q;                   // queries [q0, q0 + num_q) of this launch
+  int H_I, d_I, n_pad;             // n_pad: MMA N (16 or 32)
   int stages;
-  // Reindex: tiles are 16 pool blocks of 8 rows each
-  const int32_t* pool;
+  const int32_t* pool;             // Reindex: tiles are 16 pool blocks of 8 rows each
   int pool_blocks;
-  // outputs
-  uint32_t* keys;
+  uint32_t* keys;                  // [q][key_stride]
   int64_t key_stride;
-  uint32_t* bkeys;                 // block-max keys (Full with pool) or null
+  uint32_t* bkeys;                 // block-max keys [q][bkey_stride] (Full with pool) or null
   int64_t bkey_stride;
   int block;                       // block size for bkeys (power of two <= 32)
+  uint32_t* hist;                  // [q][kHistBins] first-digit histogram of keys
+  uint32_t* bhist;                 // same for block keys (or null)
 };
 
 struct ScoreSmem {
@@ -84,12 +100,19 @@ struct ScoreSmem {
 };
 
 template <bool kGather>
-__device__ __forceinline__ bool tile_active(const ScoreArgs& a, int q, int t, int vis) {
-  if (kGather) {
-    const int b0 = t * 16;
-    return b0 < a.pool_blocks && a.pool[(int64_t)q * a.pool_blocks + b0] >= 0;
+__device__ __forceinline__ int tiles_of(const ScoreArgs& a, int q) {
+  if (kGather) return (pool_valid(a.pool + (int64_t)q * a.pool_blocks, a.pool_blocks) + 15) / 16;
+  return (visible_of(a.seqs, q) + kTileRows - 1) / kTileRows;
+}
+
+// the row (query) of flat tile index i: the largest r with rowp[r] <= i
+__device__ __forceinline__ int find_row(const uint32_t* rowp, int n, uint32_t i) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (rowp[mid] <= i) lo = mid; else hi = mid - 1;
   }
-  return t * kTileRows < vis;
+  return lo;
 }
 
 template <bool kGather>
@@ -98,7 +121,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                  const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ ScoreSmem ss;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* status = a.seqs.status;
 
   const int halves = a.d_I >> 6;                          // 64-element K chunks
@@ -108,9 +131,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int S = a.stages;
-  const int n_items = a.num_q * a.tiles_per_q;
+  uint32_t* rowp = reinterpret_cast<uint32_t*>(base + (size_t)S * stage_bytes);   // [num_q + 1]
+  uint32_t* shist = rowp + ((a.num_q + 1 + 31) & ~31);                             // [kHistBins]
+  uint32_t* sbhist = shist + kHistBins;                                            // [kHistBins]
 
-  if (threadIdx.x == 0) {
+  // active tiles of every query, then their exclusive prefix
+  if (kGather) {
+    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = 0;
+    __syncthreads();
+    const int64_t n = (int64_t)a.num_q * a.pool_blocks;
+    const int32_t* pl = a.pool + (int64_t)a.q0 * a.pool_blocks;
+    for (int64_t b0 = 0; b0 < n; b0 += 16 * kScoreThreads) {    // 16 loads in flight
+      int32_t v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t i = b0 + j * kScoreThreads + tid;
+        v[j] = i < n ? __ldg(pl + i) : -1;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t i = b0 + j * kScoreThreads + tid;
+        if (v[j] >= 0) atomicAdd(&rowp[i / a.pool_blocks + 1], 1u);   // valid pool entries
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = (rowp[i + 1] + 15) / 16;
+  } else {
+    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles_of<kGather>(a, a.q0 + i);
+  }
+  for (int i = tid; i < 2 * kHistBins; i += kScoreThreads) shist[i] = 0;
+  if (tid == 0) {
+    rowp[0] = 0;
     for (int s = 0; s < S; ++s) { mbar_init(&ss.full[s], 1); mbar_init(&ss.empty[s], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&ss.tfull[i], 1); mbar_init(&ss.tempty[i], 4); }
     ss.abort = 0;
@@ -119,28 +170,45 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   // padding rows of the B operand (heads >= H_I) must read as zero; TMA never writes them
   for (int s = 0; s < S; ++s) {
     uint8_t* b = base + (size_t)s * stage_bytes + a_bytes;
-    for (uint32_t i = threadIdx.x * 16; i < (uint32_t)halves * b_half; i += blockDim.x * 16)
+    for (uint32_t i = tid * 16; i < (uint32_t)halves * b_half; i += kScoreThreads * 16)
       *reinterpret_cast<uint4*>(b + i) = make_uint4(0, 0, 0, 0);
   }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t carry = 0;
+    for (int b0 = 0; b0 < a.num_q; b0 += 32) {
+      const int i = b0 + lane;
+      uint32_t v = i < a.num_q ? rowp[i + 1] : 0u;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+      }
+      if (i < a.num_q) rowp[i + 1] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
   if (warp == 1) { tmem_alloc(&ss.tmem_base, a.n_pad * 2 < 32 ? 32 : a.n_pad * 2); tmem_relinquish(); }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem_base;
   volatile int* abort = &ss.abort;
+  const uint32_t total = rowp[a.num_q];
+  const uint32_t t_lo = (uint32_t)(((uint64_t)total * blockIdx.x) / gridDim.x);
+  const uint32_t t_hi = (uint32_t)(((uint64_t)total * (blockIdx.x + 1)) / gridDim.x);
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    if (lane == 0) {
+    if (lane == 0 && t_lo < t_hi) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_q);
       int stage = 0;
       uint32_t phase = 0;
-      for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
-        const int q = it / a.tiles_per_q, t = it % a.tiles_per_q;
-        const int vis = visible_of(a.seqs, q);
-        if (!tile_active<kGather>(a, q, t, vis)) continue;
+      int r = find_row(rowp, a.num_q, t_lo);
+      for (uint32_t i = t_lo; i < t_hi && !*abort; ++i) {
+        while (rowp[r + 1] <= i) ++r;
+        const int q = a.q0 + r, t = (int)(i - rowp[r]);
         if (!mbar_wait(&ss.empty[stage], phase ^ 1, abort, status)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
@@ -149,9 +217,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         int32_t blk_row[16];
         if (kGather) {
           const int32_t* pb = a.pool + (int64_t)q * a.pool_blocks + t * 16;
-          for (int i = 0; i < 16; ++i) {
-            const int j = (t * 16 + i < a.pool_blocks) ? pb[i] : -1;
-            blk_row[i] = (j >= 0) ? (int32_t)(row0 + 8 * (int64_t)j) : -1;
+          for (int k = 0; k < 16; ++k) {
+            const int j = (t * 16 + k < a.pool_blocks) ? pb[k] : -1;
+            blk_row[k] = (j >= 0) ? (int32_t)(row0 + 8 * (int64_t)j) : -1;
             if (j >= 0) bytes += (uint32_t)halves * 8 * 128;
           }
         } else {
@@ -161,9 +229,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int h = 0; h < halves; ++h) {
           tma_load_2d(sb + h * b_half, &tm_q, h * 64, q * a.H_I, &ss.full[stage]);
           if (kGather) {
-            for (int i = 0; i < 16; ++i)
-              if (blk_row[i] >= 0)
-                tma_load_2d(sa + h * (kTileRows * 128) + i * 1024, &tm_k, h * 64, blk_row[i],
+            for (int k = 0; k < 16; ++k)
+              if (blk_row[k] >= 0)
+                tma_load_2d(sa + h * (kTileRows * 128) + k * 1024, &tm_k, h * 64, blk_row[k],
                             &ss.full[stage]);
           } else {
             tma_load_2d(sa + h * (kTileRows * 128), &tm_k, h * 64,
@@ -175,14 +243,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    if (lane == 0 && t_lo < t_hi) {
       const uint32_t idesc = idesc_bf16(kTileRows, a.n_pad);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
-        const int q = it / a.tiles_per_q, t = it % a.tiles_per_q;
-        const int vis = visible_of(a.seqs, q);
-        if (!tile_active<kGather>(a, q, t, vis)) continue;
+      for (uint32_t i = t_lo; i < t_hi && !*abort; ++i) {
         if (!mbar_wait(&ss.tempty[acc], acc_phase ^ 1, abort, status)) break;
         if (!mbar_wait(&ss.full[stage], phase, abort, status)) break;
         tc_fence_after();
@@ -203,52 +268,86 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
   } else {
     // ------------------------------ epilogue (warps 2..5) ------------------------------
+    // Every epilogue warp walks every tile of the range (even after an abort) so that the
+    // named barriers of the histogram flushes always see all four warps.
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;          // entry (or slot) within the tile
+    const int etid = tid - 64;                 // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
-      const int q = it / a.tiles_per_q, t = it % a.tiles_per_q;
-      const int vis = visible_of(a.seqs, q);
-      const bool active = tile_active<kGather>(a, q, t, vis);
-      const int e = t * kTileRows + row;       // position (Full) or slot (Reindex)
-      if (!active) {
-        if (kGather && e < a.pool_blocks * 8) a.keys[(int64_t)q * a.key_stride + e] = 0u;
-        continue;
+    int hq = -1;                               // row whose histogram is being built
+    auto flush = [&](int rq) {
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      for (int b = etid; b < kHistBins; b += 128) {
+        const uint32_t v = shist[b];
+        if (v) { atomicAdd(a.hist + (int64_t)rq * kHistBins + b, v); shist[b] = 0; }
+        if (a.bhist) {
+          const uint32_t u = sbhist[b];
+          if (u) { atomicAdd(a.bhist + (int64_t)rq * kHistBins + b, u); sbhist[b] = 0; }
+        }
       }
-      if (!mbar_wait(&ss.tfull[acc], acc_phase, abort, status)) break;
-      tc_fence_after();
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+    };
+    int r = t_lo < t_hi ? find_row(rowp, a.num_q, t_lo) : 0;
+    float wr[32];                              // the current query's head weights
+    int vis = 0;
+    for (uint32_t i = t_lo; i < t_hi; ++i) {
+      while (rowp[r + 1] <= i) ++r;
+      const int q = a.q0 + r, t = (int)(i - rowp[r]);
+      if (q != hq) {
+        if (hq >= 0) flush(hq);
+        hq = q;
+        vis = visible_of(a.seqs, q);
+        const float* wq = a.w + (int64_t)q * a.H_I;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) wr[h] = h < a.H_I ? __ldg(wq + h) : 0.0f;
+      }
+      const int e = t * kTileRows + row;       // position (Full) or slot (Reindex)
+      int jpool = -1;                          // Reindex: this slot's pool block
+      if (kGather && e < a.pool_blocks * 8) jpool = __ldg(a.pool + (int64_t)q * a.pool_blocks + (e >> 3));
+      bool ok = mbar_wait(&ss.tfull[acc], acc_phase, abort, status);
+      ok = __all_sync(0xffffffffu, ok);
       float v[32];
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * a.n_pad);
-      tmem_ld16(taddr, v);
-      if (a.n_pad > 16) tmem_ld16(taddr + 16, v + 16);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ss.tempty[acc]);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * a.n_pad);
+        tmem_ld16(taddr, v);
+        if (a.n_pad > 16) tmem_ld16(taddr + 16, v + 16);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ss.tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (!ok) continue;
 
-      const float* wq = a.w + (int64_t)q * a.H_I;
       float s = 0.0f;
-      for (int h = 0; h < a.H_I; ++h) s = fmaf(__ldg(wq + h), fmaxf(v[h], 0.0f), s);
+#pragma unroll
+      for (int h = 0; h < 32; ++h)
+        if (h < a.H_I) s = fmaf(wr[h], fmaxf(v[h], 0.0f), s);
       uint32_t key = ordered_key(s);
       if (kGather) {
         if (e < a.pool_blocks * 8) {
-          const int j = a.pool[(int64_t)q * a.pool_blocks + (e >> 3)];
-          const int64_t pos = 8 * (int64_t)j + (e & 7);
-          if (j < 0 || pos >= vis) key = 0u;
+          if (jpool < 0 || 8 * (int64_t)jpool + (e & 7) >= vis) key = 0u;
           a.keys[(int64_t)q * a.key_stride + e] = key;
+          if (key) atomicAdd(&shist[key >> 21], 1u);
         }
       } else {
         if (e >= vis) key = 0u;
-        if (e < vis) a.keys[(int64_t)q * a.key_stride + e] = key;
+        if (e < vis) {
+          a.keys[(int64_t)q * a.key_stride + e] = key;
+          atomicAdd(&shist[key >> 21], 1u);
+        }
         if (a.bkeys) {
           uint32_t m = key;
           for (int o = 1; o < a.block; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-          if ((e & (a.block - 1)) == 0 && e < vis)
+          if ((e & (a.block - 1)) == 0 && e < vis) {
             a.bkeys[(int64_t)q * a.bkey_stride + e / a.block] = m;
+            atomicAdd(&sbhist[m >> 21], 1u);
+          }
         }
       }
     }
+    if (hq >= 0) flush(hq);
   }
 
   tc_fence_before();
@@ -269,175 +368,119 @@ struct SelProblem {
   int k;
   int32_t* out;
   int64_t out_stride;
-  int len_mode;       // 0: visible positions, 1: visible blocks, 2: fixed slot count
-  int block;          // len_mode 1: block size
-  int fixed_len;      // len_mode 2
+  int len_mode;         // 0: visible positions, 1: visible blocks, 2: pool slots
+  int block;            // len_mode 1: block size
   const int32_t* pool;  // len_mode 2: output = 8 * pool[slot / 8] + slot % 8
   int pool_blocks;
-  uint32_t* hist;     // [num_rows][kPasses][kHistBins]
-  uint32_t* ccnt;     // [num_rows][chunks][2]
-  int chunks;
+  const uint32_t* hist; // [rows][kHistBins]
+  uint32_t* cand;       // [rows][cand_cap] candidate positions
+  uint32_t* cand_key;   // [rows][cand_cap] their keys
+  int cand_cap;
+  uint32_t* seg;        // [rows][chunks][2]: offset, count of each chunk's candidates
+  uint32_t* fill;       // [rows] candidates appended so far
+  uint32_t* done;       // [rows] chunks finished
+  int chunks;           // grid bound on chunks per row
 };
 struct SelArgs {
   SelProblem p[2];
   Seqs seqs;
 };
 
-__device__ __forceinline__ int row_len(const SelProblem& p, const Seqs& s, int r) {
-  if (p.len_mode == 2) return p.fixed_len;
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* red);
+
+// Block-wide: entries of row r to select from.  Pool-slot rows cover the active tiles of
+// the score kernel (16 pool blocks each), never past the pool's end.
+__device__ __forceinline__ int row_len(const SelProblem& p, const Seqs& s, int r, uint32_t* red) {
+  if (p.len_mode == 2) {
+    const int32_t* pr = p.pool + (int64_t)r * p.pool_blocks;
+    uint32_t n = 0;
+    for (int i = threadIdx.x; i < p.pool_blocks; i += kSelThreads) n += pr[i] >= 0;
+    const uint32_t nv = block_sum(n, red);
+    return min(p.pool_blocks * 8, (int)((nv + 15) / 16) * kTileRows);
+  }
   const int v = visible_of(s, r);
   return p.len_mode == 0 ? v : (v + p.block - 1) / p.block;
 }
 
-constexpr int pass_shift(int p) { return p == 0 ? 21 : (p == 1 ? 10 : 0); }
-constexpr int pass_bins(int p) { return p == 2 ? 1024 : 2048; }
-
-struct Resolved {
-  uint32_t prefix;   // key bits fixed by the resolved digits
-  int krem;          // how many still to take among keys matching the prefix
-  int n_valid;       // candidate count of the row
+struct Top {
+  uint32_t b1;       // first-digit bin holding the K-th key
+  uint32_t above;    // keys in bins above b1
+  uint32_t n_valid;  // candidates of the row
+  uint32_t n_cand;   // keys in bins >= b1
   int take_all;      // n_valid <= k: every candidate is selected
 };
 
-// Block-wide: reconstruct the threshold digits of passes [0, npass) from the row's
-// histograms.  All threads return the same value.
-__device__ Resolved resolve(const uint32_t* hist_row, int k, int npass) {
-  __shared__ uint32_t warp_sum[kSelThreads / 32];
-  __shared__ Resolved res;
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  uint32_t t = 0;
+  for (int i = 0; i < kSelThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+// Block-wide: the bin of a `bins`-bin histogram h that holds the k-th largest key, with
+// the count of keys above it.  All threads return the same values.
+__device__ void find_bin(const uint32_t* h, int bins, uint32_t k, uint32_t* bin, uint32_t* above,
+                         uint32_t* red) {
+  __shared__ uint32_t s_bin, s_above;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  // total candidates = sum of the pass-0 histogram
-  uint32_t local = 0;
-  for (int b = tid; b < kHistBins; b += kSelThreads) local += hist_row[b];
-  for (int o = 16; o; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  if (lane == 0) warp_sum[wid] = local;
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t n = 0;
-    for (int i = 0; i < kSelThreads / 32; ++i) n += warp_sum[i];
-    res.n_valid = (int)n;
-    res.take_all = (int)(n <= (uint32_t)k);
-    res.prefix = 0u;
-    res.krem = k;
+  const int per = bins / kSelThreads;      // contiguous bins per thread (8 or 4)
+  uint32_t c[8];
+  uint32_t mine = 0;
+  for (int i = 0; i < per; ++i) { c[i] = h[tid * per + i]; mine += c[i]; }
+  uint32_t incl = mine;                    // sum over lanes >= mine within the warp
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += y;
   }
   __syncthreads();
-  if (res.take_all) return res;
-  for (int p = 0; p < npass; ++p) {
-    const int bins = pass_bins(p);
-    const int per = bins / kSelThreads;          // 8 or 4 bins per thread, contiguous
-    const uint32_t* h = hist_row + p * kHistBins;
-    uint32_t c[8];
-    uint32_t mine = 0;
-    for (int i = 0; i < per; ++i) { c[i] = h[tid * per + i]; mine += c[i]; }
-    // suffix sum over threads: S(t) = sum_{t' >= t} mine(t')
-    uint32_t incl = mine;                        // inclusive scan from high lanes down
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
+  if (lane == 0) red[wid] = incl;
+  __syncthreads();
+  uint32_t up = 0;
+  for (int i = wid + 1; i < kSelThreads / 32; ++i) up += red[i];
+  const uint32_t S = incl + up;            // keys in bins >= my first bin
+  const uint32_t S_next = S - mine;        // keys in bins above my range
+  if (S >= k && S_next < k) {
+    uint32_t run = S_next;
+    for (int i = per - 1; i >= 0; --i) {
+      if (run + c[i] >= k) { s_bin = tid * per + i; s_above = run; break; }
+      run += c[i];
     }
-    __syncthreads();
-    if (lane == 0) warp_sum[wid] = incl;         // lane 0 holds the warp total
-    __syncthreads();
-    uint32_t above = 0;                          // totals of warps above this one
-    for (int i = wid + 1; i < kSelThreads / 32; ++i) above += warp_sum[i];
-    const uint32_t S = incl + above;             // candidates in bins >= my first bin
-    const uint32_t krem = (uint32_t)res.krem;
-    const uint32_t S_next = S - mine;            // candidates in bins above my range
-    __syncthreads();
-    if (S >= krem && S_next < krem) {
-      uint32_t run = S_next;
-      for (int i = per - 1; i >= 0; --i) {
-        if (run + c[i] >= krem) {
-          res.prefix |= (uint32_t)(tid * per + i) << pass_shift(p);
-          res.krem = (int)(krem - run);
-          break;
-        }
-        run += c[i];
-      }
-    }
-    __syncthreads();
-  }
-  return res;
-}
-
-__device__ __forceinline__ bool matches(uint32_t key, uint32_t prefix, int npass) {
-  if (npass == 0) return true;
-  const uint32_t mask = ~((1u << pass_shift(npass - 1)) - 1u);
-  return (key & mask) == prefix;
-}
-
-template <int kPass>
-__global__ void __launch_bounds__(kSelThreads) sel_hist_kernel(const SelArgs a) {
-  const SelProblem& p = a.p[blockIdx.z];
-  const int r = blockIdx.y, c = blockIdx.x;
-  if (r >= p.num_rows || c >= p.chunks) return;
-  const int len = row_len(p, a.seqs, r);
-  const int lo = c * kSelChunk, hi = min(len, lo + kSelChunk);
-  if (lo >= hi) return;
-  uint32_t* hist_row = p.hist + (int64_t)r * kPasses * kHistBins;
-  uint32_t prefix = 0;
-  if (kPass > 0) {
-    const Resolved rs = resolve(hist_row, p.k, kPass);
-    if (rs.take_all) return;
-    prefix = rs.prefix;
-  }
-  __shared__ uint32_t h[kHistBins];
-  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) h[i] = 0;
-  __syncthreads();
-  const uint32_t* keys = p.keys + (int64_t)r * p.stride;
-  const uint32_t dmask = (uint32_t)pass_bins(kPass) - 1u;
-  for (int i = lo + threadIdx.x; i < hi; i += kSelThreads) {
-    const uint32_t key = keys[i];
-    if (key == 0u || !matches(key, prefix, kPass)) continue;
-    atomicAdd(&h[(key >> pass_shift(kPass)) & dmask], 1u);
   }
   __syncthreads();
-  uint32_t* out = hist_row + kPass * kHistBins;
-  for (int i = threadIdx.x; i < pass_bins(kPass); i += kSelThreads)
-    if (h[i]) atomicAdd(out + i, h[i]);
-}
-
-// threshold key T and how many keys equal to T to take
-__device__ __forceinline__ void threshold(const Resolved& rs, uint32_t& T, int& need_eq) {
-  if (rs.take_all) { T = 0u; need_eq = 0; }   // every key > 0 is selected
-  else { T = rs.prefix; need_eq = rs.krem; }
-}
-
-__global__ void __launch_bounds__(kSelThreads) sel_count_kernel(const SelArgs a) {
-  const SelProblem& p = a.p[blockIdx.z];
-  const int r = blockIdx.y, c = blockIdx.x;
-  if (r >= p.num_rows || c >= p.chunks) return;
-  const int len = row_len(p, a.seqs, r);
-  const int lo = c * kSelChunk, hi = min(len, lo + kSelChunk);
-  if (lo >= hi) return;
-  const Resolved rs = resolve(p.hist + (int64_t)r * kPasses * kHistBins, p.k, kPasses);
-  uint32_t T; int need_eq;
-  threshold(rs, T, need_eq);
-  const uint32_t* keys = p.keys + (int64_t)r * p.stride;
-  uint32_t gt = 0, eq = 0;
-  for (int i = lo + threadIdx.x; i < hi; i += kSelThreads) {
-    const uint32_t key = keys[i];
-    gt += (key > T);
-    eq += (key == T && key != 0u);
-  }
-  __shared__ uint32_t sg[kSelThreads / 32], se[kSelThreads / 32];
-  for (int o = 16; o; o >>= 1) {
-    gt += __shfl_xor_sync(0xffffffffu, gt, o);
-    eq += __shfl_xor_sync(0xffffffffu, eq, o);
-  }
-  if ((threadIdx.x & 31) == 0) { sg[threadIdx.x >> 5] = gt; se[threadIdx.x >> 5] = eq; }
+  *bin = s_bin;
+  *above = s_above;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t G = 0, E = 0;
-    for (int i = 0; i < kSelThreads / 32; ++i) { G += sg[i]; E += se[i]; }
-    uint32_t* cc = p.ccnt + ((int64_t)r * p.chunks + c) * 2;
-    cc[0] = G;
-    cc[1] = E;
-  }
 }
 
-// exclusive block scan of one value per thread; returns the block total in *total
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total) {
-  __shared__ uint32_t ws[kSelThreads / 32];
+// h: the row's histogram, already in shared memory
+__device__ Top resolve_top(const uint32_t* h, uint32_t k, uint32_t* red) {
+  Top tp;
+  uint32_t n = 0;
+#pragma unroll
+  for (int b = threadIdx.x; b < kHistBins; b += kSelThreads) n += h[b];
+  tp.n_valid = block_sum(n, red);
+  tp.take_all = tp.n_valid <= k;
+  if (tp.take_all) {
+    tp.b1 = 0; tp.above = 0; tp.n_cand = tp.n_valid;
+    return tp;
+  }
+  find_bin(h, kHistBins, k, &tp.b1, &tp.above, red);
+  tp.n_cand = tp.above + h[tp.b1];
+  return tp;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// exclusive block scan of one value per thread; *total receives the block total
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total, uint32_t* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint32_t x = v;
   for (int o = 1; o < 32; o <<= 1) {
@@ -445,63 +488,262 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total)
     if (lane >= o) x += y;
   }
   __syncthreads();
-  if (lane == 31) ws[wid] = x;
+  if (lane == 31) red[wid] = x;
   __syncthreads();
   uint32_t before = 0, tot = 0;
   for (int i = 0; i < kSelThreads / 32; ++i) {
-    if (i < wid) before += ws[i];
-    tot += ws[i];
+    if (i < wid) before += red[i];
+    tot += red[i];
   }
   *total = tot;
   return before + x - v;
 }
 
-__global__ void __launch_bounds__(kSelThreads) sel_write_kernel(const SelArgs a) {
-  const SelProblem& p = a.p[blockIdx.z];
-  const int r = blockIdx.y, c = blockIdx.x;
-  if (r >= p.num_rows || c >= p.chunks) return;
-  const int len = row_len(p, a.seqs, r);
-  const int lo = c * kSelChunk, hi = min(len, lo + kSelChunk);
-  int32_t* out = p.out + (int64_t)r * p.out_stride;
-  if (lo >= hi && c != 0) return;
-  const Resolved rs = resolve(p.hist + (int64_t)r * kPasses * kHistBins, p.k, kPasses);
-  if (c == 0) {  // -1 padding after the selected entries
-    const int n_sel = min(p.k, rs.n_valid);
-    for (int i = n_sel + threadIdx.x; i < p.k; i += kSelThreads) out[i] = -1;
+// Candidates of a row in ascending position order: either the per-chunk segments of the
+// list (kList) or the row's keys filtered by the first digit.
+template <bool kList>
+struct CandSource {
+  const uint32_t* keys;     // the row's keys
+  const uint32_t* cand;     // the row's list: positions
+  const uint32_t* cand_key; // and their keys
+  const uint32_t* seg;      // [chunks][2]
+  const uint32_t* pre;      // shared: exclusive prefix of segment counts [nch + 1]
+  int nch;
+  uint32_t n;               // number of candidates (list) or row length (stream)
+  uint32_t b1;
+  __device__ __forceinline__ bool pred(uint32_t key) const { return key != 0u && (key >> 21) >= b1; }
+  // position of the g-th element of the source (g < n)
+  __device__ __forceinline__ uint32_t pos_at(uint32_t g, int& c) const {
+    if constexpr (!kList) {
+      return g;
+    } else {
+      while (pre[c + 1] <= g) ++c;
+      return cand[seg[2 * c] + (g - pre[c])];
+    }
   }
-  if (lo >= hi) return;
-  uint32_t T; int need_eq;
-  threshold(rs, T, need_eq);
-  // selections of the chunks before this one
-  uint32_t gt_before = 0, eq_before = 0;
-  const uint32_t* cc = p.ccnt + (int64_t)r * p.chunks * 2;
-  for (int i = 0; i < c; ++i) { gt_before += cc[2 * i]; eq_before += cc[2 * i + 1]; }
-  const uint32_t eq_take_before = min(eq_before, (uint32_t)need_eq);
-  const uint32_t take_eq = (uint32_t)need_eq - eq_take_before;   // still to take, in order
-  // this thread's contiguous segment
-  const int per = kSelChunk / kSelThreads;
-  const int s0 = lo + threadIdx.x * per, s1 = min(hi, s0 + per);
-  const uint32_t* keys = p.keys + (int64_t)r * p.stride;
+};
+
+// Shared-memory copy of a row's candidates (key, position), in position order.
+struct StagedSource {
+  const uint32_t* keys;     // shared
+  const uint32_t* pos;      // shared
+  uint32_t n;
+  __device__ __forceinline__ bool pred(uint32_t) const { return true; }
+  __device__ __forceinline__ uint32_t key_at(uint32_t g, int&) const { return keys[g]; }
+  __device__ __forceinline__ uint32_t pos_at_ordered(uint32_t g, int&) const { return pos[g]; }
+};
+template <bool kList>
+struct GlobalSource {
+  CandSource<kList> s;
+  uint32_t n;
+  __device__ __forceinline__ bool pred(uint32_t key) const { return s.pred(key); }
+  // the cursor c only moves forward, so a caller walks g in increasing order
+  __device__ __forceinline__ uint32_t pos_at_ordered(uint32_t g, int& c) const { return s.pos_at(g, c); }
+  __device__ __forceinline__ uint32_t key_at(uint32_t g, int& c) const {
+    if constexpr (kList) {
+      const uint32_t i = s.pos_at(g, c), cc = (uint32_t)c;   // advances the cursor
+      (void)i;
+      return s.cand_key[s.seg[2 * cc] + (g - s.pre[cc])];
+    } else {
+      return s.keys[g];
+    }
+  }
+};
+
+// Exact selection of the row's Top-K from its candidates (any source in position order).
+template <class Src>
+__device__ void final_select(const SelProblem& p, int r, const Top& tp, const Src& src,
+                             uint32_t* red, uint32_t* hsm) {
+  const int tid = threadIdx.x;
+  const uint32_t k = (uint32_t)p.k;
+  int32_t* out = p.out + (int64_t)r * p.out_stride;
+  const uint32_t n_sel = min(k, tp.n_valid);
+  for (uint32_t i = n_sel + tid; i < k; i += kSelThreads) out[i] = -1;
+  if (n_sel == 0) return;
+  // threshold key T: keys > T are taken, and the first need_eq keys equal to T
+  uint32_t T = 0u, need_eq = 0u;
+  if (!tp.take_all) {
+    uint32_t krem = n_sel - tp.above;      // still to take from bin b1
+    uint32_t prefix = tp.b1 << 21;
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      const int bins = pass == 0 ? 2048 : 1024;
+      const uint32_t pmask = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;
+      for (int b = tid; b < bins; b += kSelThreads) hsm[b] = 0;
+      __syncthreads();
+      int c = 0;
+      for (uint32_t g = tid; g < src.n; g += kSelThreads) {
+        const uint32_t key = src.key_at(g, c);
+        if (key != 0u && (key & pmask) == prefix) atomicAdd(&hsm[(key >> shift) & (bins - 1)], 1u);
+      }
+      __syncthreads();
+      uint32_t bin, above;
+      find_bin(hsm, bins, krem, &bin, &above, red);
+      krem -= above;
+      prefix |= bin << shift;
+    }
+    T = prefix;
+    need_eq = krem;
+  }
+  // ordered write: each thread a contiguous run of the source
+  const uint32_t per = (src.n + kSelThreads - 1) / kSelThreads;
+  const uint32_t g0 = min(src.n, tid * per), g1 = min(src.n, g0 + per);
   uint32_t my_gt = 0, my_eq = 0;
-  for (int i = s0; i < s1; ++i) {
-    const uint32_t key = keys[i];
-    my_gt += (key > T);
-    my_eq += (key == T && key != 0u);
+  int c = 0;
+  for (uint32_t g = g0; g < g1; ++g) {
+    const uint32_t key = src.key_at(g, c);
+    if (!src.pred(key)) continue;
+    my_gt += key > T;
+    my_eq += (key == T);
   }
   uint32_t tot;
-  const uint32_t eq_rank = block_excl_scan(my_eq, &tot);   // eq keys before my segment
-  const uint32_t my_take_eq = eq_rank >= take_eq ? 0u : min(my_eq, take_eq - eq_rank);
-  const uint32_t pos0 = block_excl_scan(my_gt + my_take_eq, &tot);
-  uint32_t o = gt_before + eq_take_before + pos0, taken_eq = 0;
-  for (int i = s0; i < s1; ++i) {
-    const uint32_t key = keys[i];
+  const uint32_t eq_rank = block_excl_scan(my_eq, &tot, red);
+  const uint32_t my_take = eq_rank >= need_eq ? 0u : min(my_eq, need_eq - eq_rank);
+  uint32_t o = block_excl_scan(my_gt + my_take, &tot, red);
+  uint32_t taken = 0;
+  c = 0;
+  for (uint32_t g = g0; g < g1; ++g) {
+    const uint32_t key = src.key_at(g, c);
+    if (!src.pred(key)) continue;
     bool sel = key > T;
-    if (!sel && key == T && key != 0u) { sel = taken_eq < my_take_eq; ++taken_eq; }
+    if (!sel && key == T) { sel = taken < my_take; ++taken; }
     if (sel) {
-      int32_t v = i;
-      if (p.len_mode == 2) v = 8 * p.pool[(int64_t)r * p.pool_blocks + (i >> 3)] + (i & 7);
+      const uint32_t pos = src.pos_at_ordered(g, c);
+      int32_t v = (int32_t)pos;
+      if (p.len_mode == 2) v = 8 * p.pool[(int64_t)r * p.pool_blocks + (pos >> 3)] + (int32_t)(pos & 7);
       out[o++] = v;
     }
+  }
+}
+
+constexpr int kStageCap = 12288;       // candidates staged in shared memory (96 KB)
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
+  extern __shared__ uint4 stage_raw[];      // chunk keys, later [kStageCap] keys + positions
+  uint32_t* stage_buf = reinterpret_cast<uint32_t*>(stage_raw);
+  __shared__ uint32_t red[kSelThreads / 32];
+  __shared__ uint32_t wcnt[kSelThreads / 32];
+  __shared__ uint32_t s_base;
+  __shared__ int s_last;
+  __shared__ __align__(16) uint32_t hsm[2048];
+  __shared__ uint32_t pre[kMaxListChunks + 1];
+  const SelProblem& p = a.p[blockIdx.z];
+  const int r = blockIdx.y, c = blockIdx.x;
+  if (r >= p.num_rows) return;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int len = row_len(p, a.seqs, r, red);
+  const int nch = max(1, (len + kSelChunk - 1) / kSelChunk);
+  if (c >= nch || c >= p.chunks) return;
+  const uint32_t* keys = p.keys + (int64_t)r * p.stride;
+  const int lo = c * kSelChunk, hi = min(len, lo + kSelChunk);
+  // the row's histogram and this chunk's keys, each with one round of independent loads
+  {
+    const uint4* hg = reinterpret_cast<const uint4*>(p.hist + (int64_t)r * kHistBins);
+    const uint4 h0 = hg[tid], h1 = hg[tid + kSelThreads];
+    uint4 kv[kSelChunk / 4 / kSelThreads];
+    const uint4* kg = reinterpret_cast<const uint4*>(keys + lo);
+    const int nv = (hi - lo + 3) / 4;
+#pragma unroll
+    for (int j = 0; j < kSelChunk / 4 / kSelThreads; ++j) {
+      const int u = tid + j * kSelThreads;
+      kv[j] = u < nv ? kg[u] : make_uint4(0, 0, 0, 0);
+    }
+    reinterpret_cast<uint4*>(hsm)[tid] = h0;
+    reinterpret_cast<uint4*>(hsm)[tid + kSelThreads] = h1;
+#pragma unroll
+    for (int j = 0; j < kSelChunk / 4 / kSelThreads; ++j) stage_raw[tid + j * kSelThreads] = kv[j];
+  }
+  __syncthreads();
+  const Top tp = resolve_top(hsm, (uint32_t)p.k, red);
+  const bool use_list = tp.n_cand <= (uint32_t)p.cand_cap && nch <= kMaxListChunks;
+  uint32_t* seg = p.seg + ((int64_t)r * p.chunks + c) * 2;
+  if (use_list) {
+    // append this chunk's candidates in position order: warp w owns a contiguous eighth
+    const int sub = kSelChunk / (kSelThreads / 32);
+    const int w_lo = wid * sub, w_hi = min(hi - lo, w_lo + sub);   // chunk-relative
+    auto is_cand = [&](int i) {
+      const uint32_t k = stage_buf[i];
+      return i < w_hi && k != 0u && (k >> 21) >= tp.b1;
+    };
+    uint32_t cnt = 0;
+    for (int b0 = w_lo; b0 < w_hi; b0 += 32) cnt += __popc(__ballot_sync(0xffffffffu, is_cand(b0 + lane)));
+    if (lane == 0) wcnt[wid] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t tot = 0;
+      for (int i = 0; i < kSelThreads / 32; ++i) { const uint32_t x = wcnt[i]; wcnt[i] = tot; tot += x; }
+      s_base = tot ? atomicAdd(p.fill + r, tot) : 0u;
+      seg[0] = s_base;
+      seg[1] = tot;
+    }
+    __syncthreads();
+    uint32_t o = s_base + wcnt[wid];
+    uint32_t* cand = p.cand + (int64_t)r * p.cand_cap;
+    uint32_t* cand_key = p.cand_key + (int64_t)r * p.cand_cap;
+    for (int b0 = w_lo; b0 < w_hi; b0 += 32) {
+      const int i = b0 + lane;
+      const bool pr = is_cand(i);
+      const uint32_t m = __ballot_sync(0xffffffffu, pr);
+      if (pr) {
+        const uint32_t at = o + __popc(m & lanemask_lt());
+        cand[at] = (uint32_t)(lo + i);
+        cand_key[at] = stage_buf[i];
+      }
+      o += __popc(m);
+    }
+  }
+  // the last chunk of the row to finish completes the row (no CTA waits for another)
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(p.done + r, 1u) == (uint32_t)(nch - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (use_list) {
+    // prefix of the chunks' candidate counts (4 chunks per thread)
+    const uint32_t* sg = p.seg + (int64_t)r * p.chunks * 2;
+    uint32_t cnt4[4], mine = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ci = tid * 4 + j;
+      cnt4[j] = ci < nch ? sg[2 * ci + 1] : 0u;
+      mine += cnt4[j];
+    }
+    uint32_t tot;
+    uint32_t run = block_excl_scan(mine, &tot, red);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ci = tid * 4 + j;
+      if (ci < nch) pre[ci] = run;
+      run += cnt4[j];
+    }
+    if (tid == 0) pre[nch] = tot;
+    __syncthreads();
+    CandSource<true> cs{keys, p.cand + (int64_t)r * p.cand_cap, p.cand_key + (int64_t)r * p.cand_cap,
+                        sg, pre, nch, tot, tp.b1};
+    if (cs.n <= (uint32_t)kStageCap) {
+      // one round of independent loads brings every candidate into shared memory
+      uint32_t* sk = stage_buf;
+      uint32_t* sp = stage_buf + kStageCap;
+      int cur = 0;
+#pragma unroll 4
+      for (uint32_t g = tid; g < cs.n; g += kSelThreads) {
+        while (pre[cur + 1] <= g) ++cur;
+        const uint32_t at = sg[2 * cur] + (g - pre[cur]);
+        sp[g] = cs.cand[at];
+        sk[g] = cs.cand_key[at];
+      }
+      __syncthreads();
+      StagedSource src{sk, sp, cs.n};
+      final_select(p, r, tp, src, red, hsm);
+    } else {
+      GlobalSource<true> src{cs, cs.n};
+      final_select(p, r, tp, src, red, hsm);
+    }
+  } else {
+    CandSource<false> cs{keys, nullptr, nullptr, nullptr, nullptr, nch, (uint32_t)len, tp.b1};
+    GlobalSource<false> src{cs, (uint32_t)len};
+    final_select(p, r, tp, src, red, hsm);
   }
 }
 
@@ -544,27 +786,54 @@ int device_sms() {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int cand_cap_of(int64_t row_len, int topk) {
+  const int64_t cap = std::max<int64_t>(32 * (int64_t)topk, 8192);
+  return (int)std::max<int64_t>(1, std::min<int64_t>(cap, row_len));
+}
+
+struct ProbLayout {
+  int64_t stride;
+  int chunks, cand_cap;
+  size_t keys, hist, fill, done, cand, seg;
+};
 struct WsLayout {
-  size_t keys, bkeys, hist, ccnt, total;
-  int64_t key_stride, bkey_stride;
-  int chunks_pos, chunks_blk;
+  ProbLayout p[2];
+  size_t zero_lo, zero_hi, total;
 };
 
-WsLayout layout_of(int num_q, int64_t row_len, int64_t brow_len) {
+// Workspace: status | keys (both problems) | zeroed per call: histograms, fill, done |
+// candidate lists | segment tables.
+WsLayout layout_of(int num_q, int64_t row_len, int64_t brow_len, int topk, int pool_blocks) {
   WsLayout L{};
-  L.key_stride = (row_len + 63) / 64 * 64;
-  L.bkey_stride = (brow_len + 63) / 64 * 64;
-  L.chunks_pos = (int)std::max<int64_t>(1, (row_len + kSelChunk - 1) / kSelChunk);
-  L.chunks_blk = (int)std::max<int64_t>(1, (brow_len + kSelChunk - 1) / kSelChunk);
+  const int64_t lens[2] = {row_len, brow_len};
+  const int ks[2] = {topk, std::max(pool_blocks, 1)};
   size_t off = CSA2_STATUS_BYTES;
-  L.keys = off;
-  off = align256(off + (size_t)num_q * L.key_stride * 4);
-  L.bkeys = off;
-  off = align256(off + (size_t)num_q * L.bkey_stride * 4);
-  L.hist = off;
-  off = align256(off + (size_t)2 * num_q * kPasses * kHistBins * 4);
-  L.ccnt = off;
-  off = align256(off + (size_t)num_q * (L.chunks_pos + L.chunks_blk) * 2 * 4);
+  for (int i = 0; i < 2; ++i) {
+    ProbLayout& P = L.p[i];
+    P.stride = (lens[i] + 63) / 64 * 64;
+    P.chunks = (int)std::max<int64_t>(1, (lens[i] + kSelChunk - 1) / kSelChunk);
+    P.cand_cap = cand_cap_of(lens[i], ks[i]);
+    P.keys = off;
+    off = align256(off + (size_t)num_q * P.stride * 4);
+  }
+  L.zero_lo = off;
+  for (int i = 0; i < 2; ++i) {
+    ProbLayout& P = L.p[i];
+    P.hist = off;
+    off = align256(off + (size_t)num_q * kHistBins * 4);
+    P.fill = off;
+    off = align256(off + (size_t)num_q * 4);
+    P.done = off;
+    off = align256(off + (size_t)num_q * 4);
+  }
+  L.zero_hi = off;
+  for (int i = 0; i < 2; ++i) {
+    ProbLayout& P = L.p[i];
+    P.cand = off;
+    off = align256(off + (size_t)num_q * P.cand_cap * 8);   // positions, then keys
+    P.seg = off;
+    off = align256(off + (size_t)num_q * P.chunks * 2 * 4);
+  }
   L.total = off;
   return L;
 }
@@ -580,17 +849,16 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
                         void* ws, size_t ws_bytes, cudaStream_t stream) {
   const int64_t row_len = kGather ? (int64_t)pool_blocks * 8 : max_visible;
   const int64_t brow_len = (!kGather && pool_blocks > 0) ? (max_visible + block - 1) / block : 0;
-  const WsLayout L = layout_of(num_q, row_len, brow_len);
+  const WsLayout L = layout_of(num_q, row_len, brow_len, topk, kGather ? 0 : pool_blocks);
   if (ws_bytes < L.total) return CSA2_ERR_CAPACITY;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(wsb);
-
   Seqs sq{seqs.seq_start, seqs.seq_len, q_visible, seqs.q_per_seq, max_visible, status};
 
-  // histograms start at zero
-  if (cudaMemsetAsync(wsb + L.hist, 0, L.ccnt - L.hist, stream) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (cudaMemsetAsync(wsb + L.zero_lo, 0, L.zero_hi - L.zero_lo, stream) != cudaSuccess)
+    return CSA2_ERR_CUDA;
 
-  // ---- scores ----
+  // ---- scores (+ first-digit histograms) ----
   CUtensorMap tm_k, tm_q;
   const int box_rows = kGather ? 8 : kTileRows;
   if (!make_map(&tm_k, idx_k, cap_rows, d_I, box_rows)) return CSA2_ERR_CUDA;
@@ -598,27 +866,31 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   ScoreArgs sa{};
   sa.seqs = sq;
   sa.w = w;
-  sa.num_q = num_q;
   sa.H_I = H_I;
   sa.d_I = d_I;
   sa.n_pad = H_I <= 16 ? 16 : 32;
-  sa.tiles_per_q = (int)((row_len + kTileRows - 1) / kTileRows);
   sa.pool = pool_in;
   sa.pool_blocks = pool_blocks;
-  sa.keys = reinterpret_cast<uint32_t*>(wsb + L.keys);
-  sa.key_stride = L.key_stride;
-  sa.bkeys = brow_len > 0 ? reinterpret_cast<uint32_t*>(wsb + L.bkeys) : nullptr;
-  sa.bkey_stride = L.bkey_stride;
+  sa.keys = reinterpret_cast<uint32_t*>(wsb + L.p[0].keys);
+  sa.key_stride = L.p[0].stride;
+  sa.bkeys = brow_len > 0 ? reinterpret_cast<uint32_t*>(wsb + L.p[1].keys) : nullptr;
+  sa.bkey_stride = L.p[1].stride;
   sa.block = block;
+  sa.hist = reinterpret_cast<uint32_t*>(wsb + L.p[0].hist);
+  sa.bhist = brow_len > 0 ? reinterpret_cast<uint32_t*>(wsb + L.p[1].hist) : nullptr;
   const uint32_t stage_bytes = (uint32_t)(d_I / 64) * (kTileRows * 128 + sa.n_pad * 128);
-  sa.stages = std::min<int>(8, (int)((200u * 1024u) / stage_bytes));
-  const size_t smem = (size_t)sa.stages * stage_bytes + 1024;
-  const int n_items = num_q * sa.tiles_per_q;
-  if (n_items > 0) {
-    const int sms = device_sms();
-    if (sms <= 0) return CSA2_ERR_CUDA;
-    const int grid = std::min(n_items, sms);
-    auto kern = score_kernel<kGather>;
+  const int sms = device_sms();
+  if (sms <= 0) return CSA2_ERR_CUDA;
+  auto kern = score_kernel<kGather>;
+  for (int q0 = 0; q0 < num_q; q0 += kMaxRowsPerLaunch) {
+    sa.q0 = q0;
+    sa.num_q = std::min(kMaxRowsPerLaunch, num_q - q0);
+    const size_t extra = ((size_t)(sa.num_q + 1 + 31) / 32 * 32 + 2 * kHistBins) * 4;
+    sa.stages = std::min<int>(8, (int)((216u * 1024u - extra) / stage_bytes));
+    const size_t smem = (size_t)sa.stages * stage_bytes + extra + 1024;
+    // at least one tile per CTA on average for the largest plausible work
+    const int64_t tiles_bound = (int64_t)sa.num_q * ((row_len + kTileRows - 1) / kTileRows);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_bound));
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return CSA2_ERR_CUDA;
@@ -629,50 +901,52 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   // ---- selection ----
   SelArgs sel{};
   sel.seqs = sq;
+  for (int i = 0; i < 2; ++i) {
+    SelProblem& P = sel.p[i];
+    const ProbLayout& PL = L.p[i];
+    P.keys = reinterpret_cast<const uint32_t*>(wsb + PL.keys);
+    P.stride = PL.stride;
+    P.num_rows = num_q;
+    P.hist = reinterpret_cast<const uint32_t*>(wsb + PL.hist);
+    P.cand = reinterpret_cast<uint32_t*>(wsb + PL.cand);
+    P.cand_key = P.cand + (size_t)num_q * PL.cand_cap;
+    P.cand_cap = PL.cand_cap;
+    P.seg = reinterpret_cast<uint32_t*>(wsb + PL.seg);
+    P.fill = reinterpret_cast<uint32_t*>(wsb + PL.fill);
+    P.done = reinterpret_cast<uint32_t*>(wsb + PL.done);
+    P.chunks = PL.chunks;
+  }
   SelProblem& P = sel.p[0];
-  P.keys = sa.keys;
-  P.stride = L.key_stride;
-  P.num_rows = num_q;
   P.k = topk;
   P.out = indices;
   P.out_stride = topk;
   P.len_mode = kGather ? 2 : 0;
-  P.fixed_len = (int)row_len;
   P.pool = pool_in;
   P.pool_blocks = pool_blocks;
-  P.hist = reinterpret_cast<uint32_t*>(wsb + L.hist);
-  P.ccnt = reinterpret_cast<uint32_t*>(wsb + L.ccnt);
-  P.chunks = L.chunks_pos;
   int nprob = 1;
   if (brow_len > 0) {
     SelProblem& B = sel.p[1];
-    B = P;
-    B.keys = sa.bkeys;
-    B.stride = L.bkey_stride;
     B.k = pool_blocks;
     B.out = pool_out;
     B.out_stride = pool_blocks;
     B.len_mode = 1;
     B.block = block;
-    B.pool = nullptr;
-    B.hist = P.hist + (size_t)num_q * kPasses * kHistBins;
-    B.ccnt = P.ccnt + (size_t)num_q * L.chunks_pos * 2;
-    B.chunks = L.chunks_blk;
     nprob = 2;
   }
-  const dim3 grid(std::max(L.chunks_pos, nprob == 2 ? L.chunks_blk : 1), num_q, nprob);
-  sel_hist_kernel<0><<<grid, kSelThreads, 0, stream>>>(sel);
-  sel_hist_kernel<1><<<grid, kSelThreads, 0, stream>>>(sel);
-  sel_hist_kernel<2><<<grid, kSelThreads, 0, stream>>>(sel);
-  sel_count_kernel<<<grid, kSelThreads, 0, stream>>>(sel);
-  sel_write_kernel<<<grid, kSelThreads, 0, stream>>>(sel);
+  const dim3 grid(std::max(L.p[0].chunks, nprob == 2 ? L.p[1].chunks : 1), num_q, nprob);
+  const size_t sel_smem = (size_t)2 * kStageCap * 4;
+  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sel_smem) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  select_kernel<<<grid, kSelThreads, sel_smem, stream>>>(sel);
   return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
 csa2_status_t check_common(const uint16_t* qI, const float* w, int num_q, int H_I, int d_I,
                            const uint16_t* idx_k, int64_t cap_rows, const csa2_seqs_t& seqs,
                            int topk, const int32_t* indices, const void* ws) {
-  if (num_q < 0 || H_I < 1 || H_I > 32 || (d_I != 64 && d_I != 128)) return CSA2_ERR_UNSUPPORTED;
+  if (num_q < 0 || num_q > 65535 || H_I < 1 || H_I > 32 || (d_I != 64 && d_I != 128))
+    return CSA2_ERR_UNSUPPORTED;
   if (topk < 1 || topk > 4096) return CSA2_ERR_UNSUPPORTED;
   if (cap_rows <= 0 || cap_rows > 0x7FFFFFFF) return CSA2_ERR_INVALID_ARG;
   if (seqs.num_seqs < 1 || seqs.q_per_seq < 1 ||
@@ -694,17 +968,15 @@ using namespace csa2;
 
 extern "C" size_t csa2_index_full_workspace(int32_t num_q, int32_t max_visible, int32_t topk,
                                             int32_t pool_blocks, int32_t block) {
-  (void)topk;
-  if (num_q < 0 || max_visible < 0 || block < 1) return 0;
+  if (num_q < 0 || max_visible < 0 || block < 1 || topk < 1) return 0;
   const int64_t brow = pool_blocks > 0 ? ((int64_t)max_visible + block - 1) / block : 0;
-  return layout_of(num_q, max_visible, brow).total;
+  return layout_of(num_q, max_visible, brow, topk, pool_blocks).total;
 }
 
 extern "C" size_t csa2_index_pool_workspace(int32_t num_q, int32_t pool_blocks, int32_t block,
                                             int32_t topk) {
-  (void)topk;
-  if (num_q < 0 || pool_blocks < 0 || block < 1) return 0;
-  return layout_of(num_q, (int64_t)pool_blocks * block, 0).total;
+  if (num_q < 0 || pool_blocks < 0 || block < 1 || topk < 1) return 0;
+  return layout_of(num_q, (int64_t)pool_blocks * block, 0, topk, 0).total;
 }
 
 extern "C" csa2_status_t csa2_index_full(const uint16_t* qI, const float* w, int32_t num_q,
@@ -737,8 +1009,8 @@ extern "C" csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int
                                   workspace);
   if (st != CSA2_OK || num_q == 0) return st;
   if (block != 8 || pool_blocks < 1 || pool_blocks > 8192 || !pool) return CSA2_ERR_UNSUPPORTED;
-  // visible positions inside the pool never exceed the pool's reach; the bound only
-  // clamps q_visible values that are larger than the sequence
+  // positions inside the pool are bounded by the pool; the visibility bound only clamps
+  // q_visible values that exceed the sequence
   return run_index<true>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, 0x7FFFFFFF,
                          topk, indices, pool_blocks, block, nullptr, pool, workspace, ws_bytes,
                          (cudaStream_t)stream);
