@@ -73,16 +73,8 @@ struct AttnSmem {
   float alpha[H];
   float red[4][H];
   int valid[kTile];
-  uint32_t lut[256];   // code byte -> (e2m1(low nibble), e2m1(high nibble)) as bf16x2
 };
 
-// e2m1 code (4 bits) -> value: exponent field e (2 bits, bias 1), mantissa bit m;
-// e = 0 is the subnormal m * 0.5, else (1 + m/2) * 2^(e-1)
-__device__ __forceinline__ float e2m1_val(uint32_t c) {
-  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-  const float mag = e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : 0.5f * (float)m;
-  return (c & 8u) ? -mag : mag;
-}
 // non-negative e4m3 scale byte -> value (bias 7; exponent field 0 is subnormal m * 2^-9)
 __device__ __forceinline__ float e4m3_val(uint32_t b) {
   const uint32_t e = (b >> 3) & 15u, m = b & 7u;
@@ -100,6 +92,27 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
                                    *reinterpret_cast<const __nv_bfloat162*>(&b));
   return *reinterpret_cast<const uint32_t*>(&r);
 }
+// Eight E2M1 codes (code i in bits [4i, 4i+4) of w) -> four bf16x2 words, unscaled; word k
+// holds code 2k in its low half and code 2k+1 in its high half.  Byte permutes only:
+// the 3-bit magnitude selects the bf16 high byte H and low byte L from constant tables
+//   magnitude  0     1     2     3     4     5     6     7      (value 0 .5 1 1.5 2 3 4 6)
+//   H          0x00  0x3F  0x3F  0x3F  0x40  0x40  0x40  0x40
+//   L          0x00  0x00  0x80  0xC0  0x00  0x40  0x80  0xC0
+// and the sign bit (bit 3 of a code) becomes bit 15 / 31 of its word.
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t* m) {
+  const uint32_t sel_lo = w & 0x7777u, sel_hi = (w >> 16) & 0x7777u;
+  const uint32_t h0 = __byte_perm(0x3F3F3F00u, 0x40404040u, sel_lo);
+  const uint32_t l0 = __byte_perm(0xC0800000u, 0xC0804000u, sel_lo);
+  const uint32_t h1 = __byte_perm(0x3F3F3F00u, 0x40404040u, sel_hi);
+  const uint32_t l1 = __byte_perm(0xC0800000u, 0xC0804000u, sel_hi);
+  const uint32_t se = (w & 0x08080808u) << 4;   // sign of code 2k at bit 7 of byte k
+  const uint32_t so = w & 0x80808080u;          // sign of code 2k+1 at bit 7 of byte k
+  m[0] = __byte_perm(l0, h0, 0x5140u) ^ (__byte_perm(se, so, 0x4000u) & 0x80008000u);
+  m[1] = __byte_perm(l0, h0, 0x7362u) ^ (__byte_perm(se, so, 0x5010u) & 0x80008000u);
+  m[2] = __byte_perm(l1, h1, 0x5140u) ^ (__byte_perm(se, so, 0x6020u) & 0x80008000u);
+  m[3] = __byte_perm(l1, h1, 0x7362u) ^ (__byte_perm(se, so, 0x7030u) & 0x80008000u);
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {   // 2^x (MUFU); 2^-inf = 0
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -136,48 +149,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kQChunk = H * 128;      // bytes of one Q chunk ([H rows][128 B])
   constexpr uint32_t kQBytes = kChunks * kQChunk;
   constexpr uint32_t kKVChunk = kTile * 128;  // 16 KB
-  constexpr uint32_t kTmemCols = (H + kSlabs * H) <= 32 ? 32 : ((H + kSlabs * H) <= 64 ? 64 : ((H + kSlabs * H) <= 128 ? 128 : ((H + kSlabs * H) <= 256 ? 256 : 512)));
+  constexpr uint32_t kTmemCols = (H + kSlabs * H) <= 128 ? 128 : ((H + kSlabs * H) <= 256 ? 256 : 512);
   static_assert(D % 128 == 0 && D <= 512, "shape");
   const int Hr = a.H;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ AttnSmem<H> ss;
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that the compiler keeps
+  // the shared address space (and knows these buffers do not alias `ss`)
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = base;
   uint8_t* sKV = sQ + ((kQBytes + 1023) / 1024) * 1024;
   uint8_t* sP = sKV + kChunks * kKVChunk;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+  const int hh = warp >> 2;                  // head half (softmax / epilogue columns)
   const int split = blockIdx.x, q = blockIdx.y;
   const int seq = q / a.q_per_seq;
   const int t_begin = split * a.tiles_per_split;
   const int t_end = min(a.n_tiles, t_begin + a.tiles_per_split);
   volatile int* abort = &ss.abort;
 
+  // Q goes out first: barrier init, then its TMA, by one thread
   if (tid == 0) {
     mbar_init(&ss.bar_q, 1);
     mbar_init(&ss.bar_s, 1);
     mbar_init(&ss.bar_o, 1);
     ss.abort = 0;
     fence_barrier_init();
-  }
-  if (tid < H) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
-  ss.lut[tid] = pack_bf16(e2m1_val(tid & 15u), e2m1_val((uint32_t)tid >> 4));
-  if (Hr < H) {  // rows of padding heads must read as zero; TMA writes rows < Hr only
-    for (uint32_t i = tid * 16; i < kQBytes; i += kThreads * 16)
-      *reinterpret_cast<uint4*>(sQ + i) = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-  }
-  if (warp == 0) { tmem_alloc(&ss.tmem_base, kTmemCols); tmem_relinquish(); }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = ss.tmem_base;
-  const uint32_t tS = tmem;                  // S^T: columns [0, H)
-  const uint32_t tO = tmem + H;              // O^T slab j: columns [H + jH, H + (j+1)H)
-
-  if (tid == 0) {
     tma_prefetch_desc(&tm_q);
     mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * Hr * 128);
     for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunk, &tm_q, c * 64, q * Hr, &ss.bar_q);
@@ -190,44 +190,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_win = (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0);
   const int64_t wrow0 = a.swa_start[seq] + w0;
 
+  // gather geometry: kParts threads per row, each covering 32 columns (4 units of 8 bf16)
+  constexpr int kParts = D / 32;
+  constexpr int kRowsPerIter = kThreads / kParts;
+  constexpr int kIters = kTile / kRowsPerIter;
+  // consecutive threads take consecutive rows: the 8 threads of a quarter warp then store
+  // to 8 different rows, whose 128-byte swizzle puts their 16-byte units in 8 bank groups
+  const int rsub = tid % kRowsPerIter;
+  const int part = tid / kRowsPerIter;
+  int kind[kIters];                          // 0 invalid, 1 FP4 row, 2 window row
+  int32_t gidx[kIters];                      // FP4: sequence position; window: offset in window
+  // Phase 1 of a tile's gather: slot -> source (the index load is only issued here).
+  auto issue_slots = [&](int t) {
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int slot = t * kTile + it * kRowsPerIter + rsub;
+      kind[it] = 0;
+      gidx[it] = 0;
+      if (slot < a.topk) {
+        gidx[it] = __ldg(a.indices + (int64_t)q * a.topk + slot);
+        kind[it] = 1;
+      } else if (slot - a.topk < n_win) {
+        gidx[it] = slot - a.topk;
+        kind[it] = 2;
+      }
+    }
+  };
+  if (t_begin < t_end) issue_slots(t_begin);
+
+  if (tid < H) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
+  if (Hr < H) {  // rows of padding heads must read as zero; TMA writes rows < Hr only
+    const uint32_t pad = (uint32_t)(H - Hr) * 128;
+    for (uint32_t i = tid * 16; i < kChunks * pad; i += kThreads * 16) {
+      const uint32_t c = i / pad, o = i % pad;
+      *reinterpret_cast<uint4*>(sQ + c * kQChunk + (uint32_t)Hr * 128 + o) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) { tmem_alloc(&ss.tmem_base, kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss.tmem_base;
+  const uint32_t tS = tmem;                  // S^T: columns [0, H)
+  const uint32_t tO = tmem + H;              // O^T slab j: columns [H + jH, H + (j+1)H)
+  const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+
   const uint32_t idesc_s = idesc_bf16(kTile, H);
   const uint32_t idesc_o = idesc_bf16(kTile, H, true, true);
   uint32_t ph_s = 0, ph_o = 0;
   bool q_ready = false, o_init = false, o_pending = false;
 
-  for (int t = t_begin; t < t_end && !*abort; ++t) {
+  for (int t = t_begin; t < t_end; ++t) {
+    if (t != t_begin) issue_slots(t);        // in flight while the previous O^T finishes
     // the previous tile's O^T MMA must be done before its KV / P buffers are rewritten
     if (o_pending) {
-      if (!mbar_wait(&ss.bar_o, ph_o, abort, a.status)) break;
+      const bool ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status);
+      if (__syncthreads_or(!ok)) break;
       ph_o ^= 1;
       o_pending = false;
       tc_fence_after();
     }
     // ------------------------------ gather ------------------------------
-    // Three phases so that every global load of the tile is in flight at once: the slot
-    // indices, then the rows (FP4 codes + scales into registers, window rows by cp.async
-    // straight to shared memory), then dequantisation and the swizzled shared stores.
-    constexpr int kParts = D / 32;                 // 32-column parts per row
-    constexpr int kRowsPerIter = kThreads / kParts;
-    constexpr int kIters = kTile / kRowsPerIter;
-    const int part = tid % kParts;
-    const int rsub = tid / kParts;
-    int kind[kIters];                              // 0 invalid, 1 FP4 row, 2 window row
-    int64_t grow[kIters];
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int slot = t * kTile + it * kRowsPerIter + rsub;
-      kind[it] = 0;
-      grow[it] = 0;
-      if (slot < a.topk) {
-        const int p = __ldg(a.indices + (int64_t)q * a.topk + slot);
-        grow[it] = p;                              // resolved below, after all loads issue
-        kind[it] = 1;
-      } else if (slot - a.topk < n_win) {
-        grow[it] = wrow0 + (slot - a.topk);
-        kind[it] = 2;
-      }
-    }
+    // Phase 2: the rows -- FP4 codes + scales into registers, window rows by cp.async
+    // straight to shared memory; phase 3: dequantise (LUT + exact bf16 multiply) and store
+    // into the 128-byte-swizzled [128 keys x D] tile.
     uint4 cw[kIters];
     uint32_t sc[kIters];
 #pragma unroll
@@ -235,23 +262,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = it * kRowsPerIter + rsub;
       uint8_t* row_smem = sKV + r * 128;
       if (kind[it] == 1) {
-        const int p = (int)grow[it];
+        const int p = gidx[it];
         if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
-          grow[it] = row0 + p;
-          cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow[it] * (D / 2) + part * 16));
-          sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow[it] * (D / 16) + part * 2));
+          const int64_t grow = row0 + p;
+          cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
+          sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
         } else {
           if (p >= slen || p < -1) report(a.status, CSA2_ERR_INVALID_ARG);
           else if (p >= 0) report(a.status, CSA2_ERR_CAPACITY);
           kind[it] = 0;
         }
       } else if (kind[it] == 2) {
-        if (grow[it] >= 0 && grow[it] < a.swa_rows) {
+        const int64_t grow = wrow0 + gidx[it];
+        if (grow >= 0 && grow < a.swa_rows) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int u = 4 * part + i;
             cp_async16(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4),
-                       a.swa + grow[it] * D + u * 8);
+                       a.swa + grow * D + u * 8);
           }
         } else {
           report(a.status, CSA2_ERR_CAPACITY);
@@ -273,8 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t s2 = i < 2 ? s02 : s12;
           uint4 o;
           uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+          e2m1x8_to_bf16(w4[i], ow);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ss.lut[(w4[i] >> (8 * k)) & 0xFFu], s2);
+          for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ow[k], s2);
           const int u = 4 * part + i;
           *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
         }
@@ -298,156 +327,154 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!q_ready) { ok = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = ok; }
       if (ok) {
         tc_fence_after();
-        const uint32_t kv = smem_u32(sKV), qs = smem_u32(sQ);
+        const uint64_t kv_desc_k = sdesc_sw128(smem_u32(sKV), 16, 1024);   // KV as K-major A
+        const uint64_t q_desc_k = sdesc_sw128(smem_u32(sQ), 16, 1024);     // Q as K-major B
 #pragma unroll 4
         for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(kv + (k >> 2) * kKVChunk + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(qs + (k >> 2) * kQChunk + (k & 3) * 32, 16, 1024);
-          umma_bf16(tS, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)(k >> 2) * kKVChunk + (k & 3) * 32;
+          const uint32_t qoff = (uint32_t)(k >> 2) * kQChunk + (k & 3) * 32;
+          umma_bf16(tS, kv_desc_k + (off >> 4), q_desc_k + (qoff >> 4), idesc_s, k > 0 ? 1u : 0u);
         }
         umma_commit(&ss.bar_s);
       }
     }
 
-    // ------------------------------ softmax (warps 0-3) ------------------------------
-    if (warp < 4) {
-      const int r = warp * 32 + lane;             // key row = TMEM lane
-      if (tid == 0) ss.rescale = 0;
-      float v[H];
-      bool ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
+    // ------------------------------ softmax (all 8 warps) ------------------------------
+    // warp w: keys of TMEM lane quadrant (w & 3), heads [32 * (w >> 2), +32)
+    const int r = quad * 32 + lane;               // key row = TMEM lane
+    const int h0 = hh * 32;
+    float v[32];
+    bool ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
+    ok = __syncthreads_and(ok);
+    ph_s ^= 1;
+    if (!ok) break;
+    tc_fence_after();
+    tmem_ld32(tS + lane_base + h0, tS + lane_base + h0 + 16, v);
+    {
+      const bool valid = ss.valid[r] != 0;
 #pragma unroll
-        for (int c = 0; c < H; c += 16) tmem_ld16(tS + ((uint32_t)(warp * 32) << 16) + c, v + c);
-        const bool valid = ss.valid[r] != 0;
+      for (int h = 0; h < 32; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
+      float red[32];
 #pragma unroll
-        for (int h = 0; h < H; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
-        // per-head tile maximum
-        float red[H];
-#pragma unroll
-        for (int h = 0; h < H; ++h) red[h] = v[h];
-        reduce_scatter_step<H, 16, true>(red, lane);
-        constexpr int kOwn = H / 32;
-#pragma unroll
-        for (int i = 0; i < kOwn; ++i) ss.red[warp][kOwn * lane + i] = red[i];
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (ok) {
-        if (tid < H) {
-          const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
-          ss.alpha[tid] = mt;                     // stash the tile max
-          if (mt > ss.m_ref[tid] + kRescaleLog2) ss.rescale = 1;
-        }
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int need = ss.rescale;
-      if (ok && need) {
-        // move every head's reference max up to its running max; O and l scale by alpha
-        if (tid < H) {
-          const float mo = ss.m_ref[tid];
-          const float mn = fmaxf(mo, ss.alpha[tid]);
-          const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
-          ss.alpha[tid] = al;
-          ss.l_acc[tid] *= al;
-          ss.m_ref[tid] = mn;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (o_init) {
-#pragma unroll
-          for (int j = 0; j < kSlabs; ++j) {
-#pragma unroll
-            for (int c = 0; c < H; c += 16) {
-              float o[16];
-              const uint32_t ta = tO + ((uint32_t)(warp * 32) << 16) + j * H + c;
-              tmem_ld16(ta, o);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] *= ss.alpha[c + i];
-              tmem_st16(ta, o);
-            }
-          }
-          tmem_wait_st();
-        }
-      }
-      if (ok) {
-        // p = 2^(s - m_ref), rounded to bf16; P row r = [heads] (MN-major operand)
-        float psum[H];
-#pragma unroll
-        for (int u = 0; u < H / 8; ++u) {
-          uint4 pk;
-          uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int h = 8 * u + 2 * k;
-            const float p0 = fast_exp2(v[h] - ss.m_ref[h]);
-            const float p1 = fast_exp2(v[h + 1] - ss.m_ref[h + 1]);
-            pw[k] = pack_bf16(p0, p1);
-            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&pw[k]);
-            const float2 f = __bfloat1622float2(b);
-            psum[h] = f.x;
-            psum[h + 1] = f.y;
-          }
-          *reinterpret_cast<uint4*>(sP + r * 128 + ((u ^ (r & 7)) << 4)) = pk;
-        }
-        reduce_scatter_step<H, 16, false>(psum, lane);
-        constexpr int kOwn = H / 32;
-#pragma unroll
-        for (int i = 0; i < kOwn; ++i) ss.red[warp][kOwn * lane + i] = psum[i];
-        fence_proxy_async_smem();
-        tc_fence_before();
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (ok) {
-        if (tid < H) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
-        // ------------------------------ O^T += V^T . P^T ------------------------------
-        if (tid == 0) {
-          tc_fence_after();
-          const uint32_t kv = smem_u32(sKV), ps = smem_u32(sP);
-#pragma unroll 1
-          for (int j = 0; j < kSlabs; ++j) {
-#pragma unroll 4
-            for (int k = 0; k < kTile / 16; ++k) {
-              const uint64_t ad = sdesc_sw128(kv + (2 * j) * kKVChunk + k * 2048, kKVChunk, 1024);
-              const uint64_t bd = sdesc_sw128(ps + k * 2048, 8192, 1024);
-              umma_bf16(tO + j * H, ad, bd, idesc_o, (o_init || k > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit(&ss.bar_o);
-        }
-      }
-      ph_s ^= 1;
+      for (int h = 0; h < 32; ++h) red[h] = v[h];
+      reduce_scatter_step<32, 16, true>(red, lane);     // lane holds head h0 + lane
+      ss.red[quad][h0 + lane] = red[0];
+    }
+    if (tid == 0) ss.rescale = 0;
+    __syncthreads();
+    if (tid < H) {
+      const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
+      ss.alpha[tid] = mt;                          // stash the tile max
+      if (mt > ss.m_ref[tid] + kRescaleLog2) ss.rescale = 1;
     }
     __syncthreads();
+    if (ss.rescale) {
+      // move every head's reference max up to its running max; O and l scale by alpha
+      if (tid < H) {
+        const float mo = ss.m_ref[tid];
+        const float mn = fmaxf(mo, ss.alpha[tid]);
+        const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+        ss.alpha[tid] = al;
+        ss.l_acc[tid] *= al;
+        ss.m_ref[tid] = mn;
+      }
+      __syncthreads();
+      if (o_init) {
+        float al[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) al[i] = ss.alpha[h0 + i];
+#pragma unroll 1
+        for (int j = 0; j < kSlabs; ++j) {
+          float o[32];
+          const uint32_t ta = tO + lane_base + j * H + h0;
+          tmem_ld32(ta, ta + 16, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= al[i];
+          tmem_st16(ta, o);
+          tmem_st16(ta + 16, o + 16);
+        }
+        tmem_wait_st();
+      }
+    }
+    {
+      // p = 2^(s - m_ref), rounded to bf16; P row r = [heads] (the MN-major B operand)
+      // (v is overwritten with the bf16-rounded p for the per-head sums)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint4 pk;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int h = 8 * u + 2 * k;
+          const float p0 = fast_exp2(v[h] - ss.m_ref[h0 + h]);
+          const float p1 = fast_exp2(v[h + 1] - ss.m_ref[h0 + h + 1]);
+          pw[k] = pack_bf16(p0, p1);
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[k]));
+          v[h] = f.x;
+          v[h + 1] = f.y;
+        }
+        const int unit = 4 * hh + u;
+        *reinterpret_cast<uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
+      }
+      reduce_scatter_step<32, 16, false>(v, lane);
+      ss.red[quad][h0 + lane] = v[0];
+      fence_proxy_async_smem();
+      tc_fence_before();
+    }
+    __syncthreads();
+    if (tid < H) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
+    // ------------------------------ O^T += V^T . P^T ------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t kv_desc_mn = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);  // V^T, MN-major A
+      const uint64_t p_desc_mn = sdesc_sw128(smem_u32(sP), 8192, 1024);        // P^T, MN-major B
+#pragma unroll 1
+      for (int j = 0; j < kSlabs; ++j) {
+#pragma unroll 4
+        for (int k = 0; k < kTile / 16; ++k) {
+          const uint32_t off = (uint32_t)(2 * j) * kKVChunk + k * 2048;
+          umma_bf16(tO + j * H, kv_desc_mn + (off >> 4), p_desc_mn + ((uint32_t)(k * 2048) >> 4),
+                    idesc_o, (o_init || k > 0) ? 1u : 0u);
+        }
+      }
+      umma_commit(&ss.bar_o);
+    }
     o_init = true;
     o_pending = true;
   }
 
   // ------------------------------ epilogue ------------------------------
-  if (o_pending) {
-    if (mbar_wait(&ss.bar_o, ph_o, abort, a.status)) tc_fence_after();
+  bool done_ok = !*abort;
+  if (o_pending) done_ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status) && done_ok;
+  done_ok = __syncthreads_and(done_ok);
+  tc_fence_after();
+  const bool partial = a.nsplit > 1;
+  if (tid < H) {  // reciprocal of l for the normalised (unsplit) output
+    const float l = ss.l_acc[tid];
+    ss.alpha[tid] = (!partial && l > 0.0f) ? 1.0f / l : 1.0f;
   }
   __syncthreads();
-  // The KV tile is free once the last O^T MMA has completed: stage O (normalised unless
-  // partial) there as [head][D] fp32, then copy it out with 16-byte stores.
-  const bool partial = a.nsplit > 1;
+  // The KV tile is free once the last O^T MMA has completed: stage O there as [head][D]
+  // fp32, then copy it out with 16-byte stores.
   float* so = reinterpret_cast<float*>(sKV);        // [Hr][D] (Hr * D * 4 <= 128 KB)
-  if (warp < 4 && !*abort) {
+  if (done_ok) {
+    const int hbase = hh * 32;
+    float oscale[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      oscale[i] = (o_init && ss.l_acc[hbase + i] > 0.0f) ? ss.alpha[hbase + i] : 0.0f;
 #pragma unroll 1
     for (int j = 0; j < kSlabs; ++j) {
-      const int d = j * 128 + warp * 32 + lane;
-#pragma unroll 1
-      for (int c = 0; c < H; c += 16) {
-        float o[16];
-        if (o_init) tmem_ld16(tO + ((uint32_t)(warp * 32) << 16) + j * H + c, o);
+      const int d = j * 128 + quad * 32 + lane;
+      float o[32];
+      if (o_init) {
+        const uint32_t ta = tO + lane_base + j * H + hbase;
+        tmem_ld32(ta, ta + 16, o);
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (c + i < Hr) {
-            const float l = ss.l_acc[c + i];
-            float val = o_init ? o[i] : 0.0f;
-            if (!partial) val = (l > 0.0f) ? val / l : 0.0f;
-            so[(c + i) * D + d] = val;
-          }
-        }
+      for (int i = 0; i < 32; ++i) {
+        const int h = hbase + i;
+        if (h < Hr) so[h * D + d] = o_init ? o[i] * oscale[i] : 0.0f;
       }
     }
     if (tid < Hr) {
@@ -462,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  if (!*abort) {
+  if (done_ok) {
     float4* dst4 = reinterpret_cast<float4*>(partial ? a.part_o + (((int64_t)q * a.nsplit + split) * Hr) * D
                                                      : a.out + (int64_t)q * Hr * D);
     const float4* src4 = reinterpret_cast<const float4*>(so);

@@ -128,8 +128,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const uint32_t a_bytes = (uint32_t)halves * kTileRows * 128;
   const uint32_t b_half = (uint32_t)a.n_pad * 128;
   const uint32_t stage_bytes = a_bytes + (uint32_t)halves * b_half;
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that the compiler keeps
+  // the shared address space (and knows these buffers do not alias `ss`)
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = a.stages;
   uint32_t* rowp = reinterpret_cast<uint32_t*>(base + (size_t)S * stage_bytes);   // [num_q + 1]
   uint32_t* shist = rowp + ((a.num_q + 1 + 31) & ~31);                             // [kHistBins]
