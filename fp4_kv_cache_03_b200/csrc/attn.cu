@@ -449,6 +449,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   done_ok = __syncthreads_and(done_ok);
   tc_fence_after();
   const bool partial = a.nsplit > 1;
+  if (partial) {
+    // Split query: write this CTA's unnormalised O (relative to m_ref) as [D][Hr] rows,
+    // straight from TMEM (16-byte stores of 32 heads per thread), plus (m, l) per head.
+    if (done_ok) {
+      float* po = a.part_o + ((int64_t)q * a.nsplit + split) * D * Hr;
+      const int hbase = hh * 32;
+#pragma unroll 1
+      for (int j = 0; j < kSlabs; ++j) {
+        const int d = j * 128 + quad * 32 + lane;
+        float o[32];
+        if (o_init) {
+          const uint32_t ta = tO + lane_base + j * H + hbase;
+          tmem_ld32(ta, ta + 16, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.0f;
+        }
+        float* row = po + (int64_t)d * Hr + hbase;
+        if (hbase + 32 <= Hr && (Hr & 3) == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(row + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (hbase + i < Hr) row[i] = o[i];
+        }
+      }
+      if (tid < Hr) {
+        const float m = ss.m_ref[tid], l = ss.l_acc[tid];
+        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + tid) * 2;
+        ml[0] = (o_init && l > 0.0f) ? m : -INFINITY;
+        ml[1] = o_init ? l : 0.0f;
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+    return;
+  }
   if (tid < H) {  // reciprocal of l for the normalised (unsplit) output
     const float l = ss.l_acc[tid];
     ss.alpha[tid] = (!partial && l > 0.0f) ? 1.0f / l : 1.0f;
@@ -505,29 +548,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// merge the split partials of one (query, head): weights 2^(m_s - M)
-template <int D>
-__global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a, int H) {
-  const int q = blockIdx.x, h = blockIdx.y;
+// Merge of the split partials of one query over a 32-dim block: per head the weights
+// 2^(m_s - M) / L, M = max_s m_s, L = sum_s 2^(m_s - M) l_s; partials are [D][H] rows, so the
+// block is read with consecutive threads on consecutive heads and transposed through
+// shared memory for the [H][D] output.
+constexpr int kMergeD = 8;               // output dims per merge CTA
+constexpr int kMaxSplit = 16;
+__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a, int H, int D) {
+  __shared__ float wgt[kMaxSplit][kN];
+  __shared__ float tile[kN][kMergeD + 1];
+  const int q = blockIdx.x, d0 = blockIdx.y * kMergeD, tid = threadIdx.x;
   const int ns = a.nsplit;
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.part_ml[(((int64_t)q * ns + s) * H + h) * 2]);
-  float L = 0.0f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int d = threadIdx.x * 4;
-  for (int s = 0; s < ns; ++s) {
-    const float* ml = a.part_ml + (((int64_t)q * ns + s) * H + h) * 2;
-    if (ml[0] == -INFINITY) continue;
-    const float wgt = exp2f(ml[0] - M);
-    L += wgt * ml[1];
-    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (((int64_t)q * ns + s) * H + h) * D + d);
-    acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
+  // partial values first: every load of this thread in flight at once
+  const float* base = a.part_o + (int64_t)q * ns * D * H + (int64_t)d0 * H;
+  const int n_el = kMergeD * H;          // <= 512: two per thread
+  float v[2][kMaxSplit];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = tid + 256 * k;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s)
+      v[k][s] = (e < n_el && s < ns) ? __ldg(base + (int64_t)s * D * H + e) : 0.0f;
   }
-  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-  *reinterpret_cast<float4*>(a.out + ((int64_t)q * H + h) * D + d) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (a.lse && threadIdx.x == 0)
-    a.lse[(int64_t)q * H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  if (tid < H) {
+    const float* ml = a.part_ml + (int64_t)q * ns * H * 2;
+    float m[kMaxSplit], l[kMaxSplit];
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) {
+      m[s] = s < ns ? ml[(s * H + tid) * 2] : -INFINITY;
+      l[s] = s < ns ? ml[(s * H + tid) * 2 + 1] : 0.0f;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) M = fmaxf(M, m[s]);
+    float L = 0.0f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) {
+      const float w = (m[s] == -INFINITY) ? 0.0f : exp2f(m[s] - M);
+      wgt[s][tid] = w;
+      L += w * l[s];
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) wgt[s][tid] *= inv;
+    if (a.lse && blockIdx.y == 0)
+      a.lse[(int64_t)q * H + tid] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = tid + 256 * k;
+    if (e < n_el) {
+      const int dd = e / H, h = e - dd * H;
+      float acc = 0.0f;
+#pragma unroll
+      for (int s = 0; s < kMaxSplit; ++s) acc = fmaf(wgt[s][h], v[k][s], acc);
+      tile[h][dd] = acc;
+    }
+  }
+  __syncthreads();
+  float* out = a.out + (int64_t)q * H * D + d0;
+  for (int e = tid; e < n_el; e += 256) {
+    const int h = e / kMergeD, dd = e - h * kMergeD;
+    out[(int64_t)h * D + dd] = tile[h][dd];
+  }
 }
 
 // ---------------------------------------------------------------------------------
@@ -539,7 +623,7 @@ int n_tiles_of(int topk, int window) { return (topk + window + kTile - 1) / kTil
 
 int nsplit_of(int num_q, int n_tiles) {
   if (n_tiles <= 1) return 1;
-  return std::max(1, std::min(n_tiles, 512 / std::max(1, num_q)));
+  return std::max(1, std::min(std::min(n_tiles, kMaxSplit), 512 / std::max(1, num_q)));
 }
 
 size_t attn_smem_bytes(int D) {
@@ -571,7 +655,7 @@ cudaError_t launch(const AttnArgs& a, const CUtensorMap& tm, cudaStream_t st) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<D><<<dim3(a.nsplit, a.num_q), kThreads, smem, st>>>(tm, a);
-  if (a.nsplit > 1) attn_merge_kernel<D><<<dim3(a.num_q, a.H), D / 4, 0, st>>>(a, a.H);
+  if (a.nsplit > 1) attn_merge_kernel<<<dim3(a.num_q, D / kMergeD), 256, 0, st>>>(a, a.H, D);
   return cudaGetLastError();
 }
 
