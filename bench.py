@@ -229,9 +229,7 @@ def run_ours(args, rank, world, local_rank):
                 latest = idx
             elif L.mode == synth.FULL and li != full_li:
                 raise NotImplementedError("one Full layer per step")
-            csa2.sparse_attn(L.q, dw.kv_codes, dw.kv_scales, dw.seqs, latest, L.swa, L.swa_start,
-                             dw.q_pos, W.window, dw.scale, dw.out[li], dw.ws_attn, lse=dw.lse[li],
-                             stream=stream)
+            dw.attend(li, latest, stream=stream)
 
     graphs = []
     with torch.cuda.stream(stream):

@@ -53,10 +53,11 @@ _SIGS = {
                                   c_int64, Seqs, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                   c_void_p, c_void_p, c_size_t, c_void_p]),
     "csa2_sparse_attn_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
+    "csa2_sparse_attn_stash_bytes": (c_size_t, [c_int32, c_int32, c_int32]),
     "csa2_sparse_attn": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                    c_int64, Seqs, c_void_p, c_int32, c_void_p, c_int64, c_void_p,
-                                   c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
-                                   c_size_t, c_void_p]),
+                                   c_void_p, c_int32, c_float, c_void_p, c_void_p, c_int32,
+                                   c_void_p, c_size_t, c_void_p, c_size_t, c_void_p]),
     "csa2_status_reset": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_fetch": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_string": (ctypes.c_char_p, [c_int32]),
@@ -182,8 +183,12 @@ def sparse_attn_workspace(num_q, H, D, topk, window) -> int:
     return int(lib().csa2_sparse_attn_workspace(num_q, H, D, topk, window))
 
 
+def sparse_attn_stash_bytes(num_q, D, topk) -> int:
+    return int(lib().csa2_sparse_attn_stash_bytes(num_q, D, topk))
+
+
 def sparse_attn(q, kv_codes, kv_scales, seqs: Seqs, indices, swa_kv, swa_start, q_pos, window,
-                softmax_scale, out, ws, lse=None, stream=None):
+                softmax_scale, out, ws, lse=None, mode=MODE_FULL, stash=None, stream=None):
     num_q, H, D = q.shape
     topk = indices.shape[1] if indices is not None else 0
     assert out.dtype == torch.float32 and q_pos.dtype == torch.int64
@@ -191,6 +196,7 @@ def sparse_attn(q, kv_codes, kv_scales, seqs: Seqs, indices, swa_kv, swa_start, 
                                   kv_codes.shape[0], seqs, _p(indices), topk, _u16(swa_kv),
                                   swa_kv.shape[0] if swa_kv is not None else 0, _p(swa_start),
                                   _p(q_pos), window, float(softmax_scale), _p(out), _p(lse),
+                                  int(mode), _p(stash), stash.numel() if stash is not None else 0,
                                   _p(ws), ws.numel(), _s(stream)), "csa2_sparse_attn")
 
 

@@ -49,6 +49,9 @@ struct AttnArgs {
   const int64_t* swa_start;
   const int64_t* q_pos;
   int window;
+  int mode;                                  // csa2_mode_t
+  uint8_t* stash;                            // [num_q][n_idx_tiles][tile bytes] or null
+  int n_idx_tiles;                           // tiles holding index slots: ceil(topk / 128)
   int H;                                     // real heads (<= kN); the rest are padding
   float scale_log2;                          // softmax_scale * log2(e)
   int n_tiles;                               // tiles of the slot list
@@ -64,7 +67,7 @@ constexpr int kN = 64;                       // MMA N: heads, padded to 64
 
 template <int H>
 struct AttnSmem {
-  uint64_t bar_q, bar_s, bar_o;
+  uint64_t bar_q, bar_s, bar_o, bar_kv;
   uint32_t tmem_base;
   int abort;
   int rescale;
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ss.bar_q, 1);
     mbar_init(&ss.bar_s, 1);
     mbar_init(&ss.bar_o, 1);
+    mbar_init(&ss.bar_kv, 1);
     ss.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
@@ -238,18 +242,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t idesc_s = idesc_bf16(kTile, H);
   const uint32_t idesc_o = idesc_bf16(kTile, H, true, true);
-  uint32_t ph_s = 0, ph_o = 0;
-  bool q_ready = false, o_init = false, o_pending = false;
+  uint32_t ph_s = 0, ph_o = 0, ph_kv = 0;
+  bool q_ready = false, o_init = false, o_pending = false, store_pending = false;
+  constexpr uint32_t kTileBytes = kChunks * kKVChunk;
 
   for (int t = t_begin; t < t_end; ++t) {
+    // Reuse with a stash: this tile's selected rows come back as the bf16 tile a Full /
+    // Reindex call stored; Full / Reindex with a stash store their tile after the gather.
+    const bool stash_tile = a.stash != nullptr && t < a.n_idx_tiles;
+    const bool from_stash = stash_tile && a.mode == CSA2_MODE_REUSE;
+    const bool to_stash = stash_tile && a.mode != CSA2_MODE_REUSE;
+    uint8_t* stile = stash_tile ? a.stash + ((int64_t)q * a.n_idx_tiles + t) * kTileBytes : nullptr;
     if (t != t_begin) issue_slots(t);        // in flight while the previous O^T finishes
     // the previous tile's O^T MMA must be done before its KV / P buffers are rewritten
+    if (store_pending && tid == 0) bulk_wait_read();
     if (o_pending) {
       const bool ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status);
       if (__syncthreads_or(!ok)) break;
       ph_o ^= 1;
       o_pending = false;
       tc_fence_after();
+    } else if (store_pending) {
+      __syncthreads();
+    }
+    store_pending = false;
+    if (from_stash) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&ss.bar_kv, kTileBytes);
+        for (int c = 0; c < kChunks; ++c)
+          bulk_g2s(sKV + c * kKVChunk, stile + c * kKVChunk, kKVChunk, &ss.bar_kv);
+      }
+      const bool ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
+      ph_kv ^= 1;
+      if (__syncthreads_or(!ok)) break;
     }
     // ------------------------------ gather ------------------------------
     // Phase 2: the rows -- FP4 codes + scales into registers, window rows by cp.async
@@ -264,9 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kind[it] == 1) {
         const int p = gidx[it];
         if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
-          const int64_t grow = row0 + p;
-          cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
-          sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
+          if (from_stash) {
+            kind[it] = 3;                          // row already in the tile (from the stash)
+          } else {
+            const int64_t grow = row0 + p;
+            cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
+            sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
+          }
         } else {
           if (p >= slen || p < -1) report(a.status, CSA2_ERR_INVALID_ARG);
           else if (p >= 0) report(a.status, CSA2_ERR_CAPACITY);
@@ -319,6 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait_all();
     fence_proxy_async_smem();
     const int any = __syncthreads_or(ss.valid[tid & (kTile - 1)]);
+    if (to_stash) {                            // keep the dequantised tile for Reuse layers
+      if (tid == 0) {
+        for (int c = 0; c < kChunks; ++c) bulk_s2g(stile + c * kKVChunk, sKV + c * kKVChunk, kKVChunk);
+        bulk_commit();
+      }
+      store_pending = true;                    // uniform: every thread takes the same branches
+    }
     if (!any) continue;
 
     // ------------------------------ S^T = KV . Q^T ------------------------------
@@ -444,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ------------------------------ epilogue ------------------------------
+  if (store_pending && tid == 0) bulk_wait_read();
   bool done_ok = !*abort;
   if (o_pending) done_ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status) && done_ok;
   done_ok = __syncthreads_and(done_ok);
@@ -664,6 +701,11 @@ cudaError_t launch(const AttnArgs& a, const CUtensorMap& tm, cudaStream_t st) {
 
 using namespace csa2;
 
+extern "C" size_t csa2_sparse_attn_stash_bytes(int32_t num_q, int32_t D, int32_t topk) {
+  if (num_q < 0 || D < 1 || topk < 0) return 0;
+  return (size_t)num_q * ((topk + kTile - 1) / kTile) * (size_t)D * 256;
+}
+
 extern "C" size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
                                              int32_t window) {
   if (num_q < 0 || H < 1 || D < 1 || topk < 0 || window < 0) return 0;
@@ -683,7 +725,8 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
                                           const uint16_t* swa_kv, int64_t swa_rows,
                                           const int64_t* swa_start, const int64_t* q_pos,
                                           int32_t window, float softmax_scale, float* out,
-                                          float* lse, void* workspace, size_t ws_bytes,
+                                          float* lse, csa2_mode_t mode, void* kv_stash,
+                                          size_t stash_bytes, void* workspace, size_t ws_bytes,
                                           void* stream) {
   if (num_q < 0 || topk < 0 || topk > 2048 || window < 0 || window > 1024) return CSA2_ERR_INVALID_ARG;
   if (!attn_shape_ok(H, D)) return CSA2_ERR_UNSUPPORTED;
@@ -691,6 +734,12 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
     return CSA2_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < csa2_sparse_attn_workspace(num_q, H, D, topk, window))
     return CSA2_ERR_CAPACITY;
+  if (mode != CSA2_MODE_FULL && mode != CSA2_MODE_REINDEX && mode != CSA2_MODE_REUSE)
+    return CSA2_ERR_INVALID_ARG;
+  if (kv_stash && (stash_bytes < csa2_sparse_attn_stash_bytes(num_q, D, topk) ||
+                   (reinterpret_cast<uintptr_t>(kv_stash) & 15)))
+    return kv_stash && (reinterpret_cast<uintptr_t>(kv_stash) & 15) ? CSA2_ERR_INVALID_ARG
+                                                                    : CSA2_ERR_CAPACITY;
   if (num_q == 0) return CSA2_OK;
   if ((int64_t)num_q * H > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;
   if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
@@ -707,6 +756,9 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   a.indices = indices; a.topk = topk;
   a.swa = swa_kv; a.swa_rows = swa_rows; a.swa_start = swa_start; a.q_pos = q_pos;
   a.window = window;
+  a.mode = (int)mode;
+  a.stash = static_cast<uint8_t*>(kv_stash);
+  a.n_idx_tiles = (topk + kTile - 1) / kTile;
   a.H = H;
   a.scale_log2 = softmax_scale * kLog2e;
   a.n_tiles = n_tiles_of(topk, window);

@@ -628,6 +628,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
   __shared__ int s_last;
   __shared__ __align__(16) uint32_t hsm[2048];
   __shared__ uint32_t pre[kMaxListChunks + 1];
+  __shared__ uint32_t soff[kMaxListChunks];  // list offset of each chunk's candidates
   const SelProblem& p = a.p[blockIdx.z];
   const int r = blockIdx.y, c = blockIdx.x;
   if (r >= p.num_rows) return;
@@ -708,6 +709,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
     for (int j = 0; j < 4; ++j) {
       const int ci = tid * 4 + j;
       cnt4[j] = ci < nch ? sg[2 * ci + 1] : 0u;
+      if (ci < nch) soff[ci] = sg[2 * ci];
       mine += cnt4[j];
     }
     uint32_t tot;
@@ -726,11 +728,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
       // one round of independent loads brings every candidate into shared memory
       uint32_t* sk = stage_buf;
       uint32_t* sp = stage_buf + kStageCap;
+      // each thread a contiguous run of the list; its first chunk by binary search
+      const uint32_t per = (cs.n + kSelThreads - 1) / kSelThreads;
+      const uint32_t g0 = min(cs.n, tid * per), g1 = min(cs.n, g0 + per);
       int cur = 0;
+      {
+        int lo = 0, hi = nch - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (pre[mid] <= g0) lo = mid; else hi = mid - 1;
+        }
+        cur = lo;
+      }
 #pragma unroll 4
-      for (uint32_t g = tid; g < cs.n; g += kSelThreads) {
+      for (uint32_t g = g0; g < g1; ++g) {
         while (pre[cur + 1] <= g) ++cur;
-        const uint32_t at = sg[2 * cur] + (g - pre[cur]);
+        const uint32_t at = soff[cur] + (g - pre[cur]);
         sp[g] = cs.cand[at];
         sk[g] = cs.cand_key[at];
       }

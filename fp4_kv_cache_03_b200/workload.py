@@ -37,7 +37,9 @@ class LayerInputs:
 class DeviceWorkload:
     FILL_ROWS = 65536
 
-    def __init__(self, W: synth.Workload, device="cuda", fill=True):
+    STASH_LIMIT = 256 << 20   # keep Reuse stashes for batches whose stash stays this small
+
+    def __init__(self, W: synth.Workload, device="cuda", fill=True, use_stash=True):
         self.W = W
         self.device = device
         dev = device
@@ -65,6 +67,10 @@ class DeviceWorkload:
         self.ws_pool = csa2.workspace(csa2.index_pool_workspace(
             nq, max(W.pool_blocks, 1), W.block, W.topk), dev) if self.has_pool else None
         self.ws_attn = csa2.workspace(csa2.sparse_attn_workspace(nq, W.H, W.D, W.topk, W.window), dev)
+        # dequantised selected rows of the latest Full/Reindex layer, for its Reuse layers
+        sb = csa2.sparse_attn_stash_bytes(nq, W.D, W.topk)
+        self.stash = (torch.empty(sb, dtype=torch.uint8, device=dev)
+                      if use_stash and 0 < sb <= self.STASH_LIMIT else None)
         self.pool = torch.full((nq, max(W.pool_blocks, 1)), -1, dtype=torch.int32, device=dev)
         n_idx = sum(1 for m in W.modes if m != synth.REUSE)
         self.indices = [torch.full((nq, W.topk), -1, dtype=torch.int32, device=dev)
@@ -151,10 +157,19 @@ class DeviceWorkload:
                 assert latest is not None, "a Reuse layer needs an earlier Full/Reindex layer"
             used.append(latest)
             if attention:
-                csa2.sparse_attn(L.q, self.kv_codes, self.kv_scales, self.seqs, latest, L.swa,
-                                 L.swa_start, self.q_pos, W.window, self.scale, self.out[li],
-                                 self.ws_attn, lse=self.lse[li], stream=stream)
+                self.attend(li, latest, stream)
         return used
+
+    MODES = {synth.FULL: csa2.MODE_FULL, synth.REINDEX: csa2.MODE_REINDEX, synth.REUSE: csa2.MODE_REUSE}
+
+    def attend(self, li: int, indices, stream=None):
+        """Attention of layer li with the given indices; Reuse layers read the stash the
+        latest Full/Reindex layer filled."""
+        L, W = self.layers[li], self.W
+        csa2.sparse_attn(L.q, self.kv_codes, self.kv_scales, self.seqs, indices, L.swa,
+                         L.swa_start, self.q_pos, W.window, self.scale, self.out[li],
+                         self.ws_attn, lse=self.lse[li], mode=self.MODES[L.mode],
+                         stash=self.stash, stream=stream)
 
     def status(self) -> int:
         """First device-side error recorded by any call (0 = none)."""

@@ -197,6 +197,15 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   l_j = softmax_scale * q[q][h] . row_j;  out[q][h] = sum_j softmax(l)_j row_j;
  *   lse[q][h] = log(sum_j exp(l_j)) (natural log); no rows at all gives out = 0,
  *   lse = -inf.  The two sets share one softmax; a row in both counts twice.
+ * Cross-layer reuse ([SURV] §2.2.2, [MTP] "CSA2：…": a Reuse layer takes the main KV and the
+ * latest Top-K of an earlier layer): with a non-NULL `kv_stash`,
+ *   - mode FULL or REINDEX also stores the dequantised selected rows (bf16, in the kernel's
+ *     tile layout) into kv_stash;
+ *   - mode REUSE takes the selected rows from kv_stash instead of the FP4 cache.  The
+ *     stash must hold the rows of exactly these indices for these queries, as written by
+ *     the latest FULL/REINDEX call with the same num_q, D and topk; the window rows are
+ *     always read from swa_kv.  Results equal those of a stateless call.
+ *   With kv_stash == NULL every mode reads the FP4 cache (the call is stateless).
  *   q         device bf16 [num_q][H][D]        1 <= H <= 64, D in {128, 256, 512} (other
  *             shapes return CSA2_ERR_UNSUPPORTED); base 16-byte aligned
  *   indices   device int32 [num_q][topk]       0 <= topk <= 2048
@@ -205,9 +214,13 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   q_pos     device int64 [num_q]
  *   window    0 .. 1024
  *   out       device fp32 [num_q][H][D];  lse device fp32 [num_q][H] or NULL
+ *   mode      csa2_mode_t (only used with a stash)
+ *   kv_stash  device, >= csa2_sparse_attn_stash_bytes(num_q, D, topk) bytes, 16-byte
+ *             aligned, or NULL
  *   workspace >= csa2_sparse_attn_workspace(...) bytes */
 CSA2_API size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
                                   int32_t window);
+CSA2_API size_t csa2_sparse_attn_stash_bytes(int32_t num_q, int32_t D, int32_t topk);
 CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_t H, int32_t D,
                                const uint8_t* kv_codes, const uint8_t* kv_scales,
                                int64_t cap_rows, csa2_seqs_t seqs,
@@ -216,6 +229,7 @@ CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_
                                const int64_t* swa_start, const int64_t* q_pos,
                                int32_t window, float softmax_scale,
                                float* out, float* lse,
+                               csa2_mode_t mode, void* kv_stash, size_t stash_bytes,
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------

@@ -85,9 +85,9 @@ def test_host_checks_index(L):
 
 def test_host_checks_attention(L):
     from fp4_kv_cache_03_b200 import csa2
-    def call(H=16, D=128, topk=64, window=128, ws=1 << 30):
+    def call(H=16, D=128, topk=64, window=128, ws=1 << 30, mode=0, stash=None, stash_bytes=0):
         return L.csa2_sparse_attn(FAKE, 1, H, D, FAKE, FAKE, 100, _seqs(), FAKE, topk, FAKE, 100,
-                                  FAKE, FAKE, window, 0.1, FAKE, None,
+                                  FAKE, FAKE, window, 0.1, FAKE, None, mode, stash, stash_bytes,
                                   ctypes.c_void_p(0x100000), ws, None)
     assert call(H=65) == csa2.ERR_UNSUPPORTED
     assert call(H=0) == csa2.ERR_UNSUPPORTED
@@ -95,6 +95,10 @@ def test_host_checks_attention(L):
     assert call(D=64) == csa2.ERR_UNSUPPORTED
     assert call(topk=4096) == csa2.ERR_INVALID_ARG
     assert call(ws=300) == csa2.ERR_CAPACITY
+    assert call(mode=7) == csa2.ERR_INVALID_ARG
+    assert call(stash=ctypes.c_void_p(0x200000), stash_bytes=16) == csa2.ERR_CAPACITY
+    assert call(stash=ctypes.c_void_p(0x200008), stash_bytes=1 << 30) == csa2.ERR_INVALID_ARG
+    assert L.csa2_sparse_attn_stash_bytes(1, 512, 512) == 4 * 128 * 512 * 2
 
 
 def test_device_query_without_gpu_is_harmless(L):

@@ -96,3 +96,20 @@ def test_bad_index_is_skipped_and_reported():
 
 def test_decoder_group_128k_attention():
     run_attn(synth.workload("decoder_group_128k"))
+
+
+def test_reuse_stash_equals_stateless():
+    """Reuse layers reading the stashed bf16 rows give bit-identical results to Reuse
+    layers that gather and dequantise the FP4 rows again; Reindex layers refresh it."""
+    from fp4_kv_cache_03_b200.workload import DeviceWorkload
+    W = small_workload(lengths=(3000, 9000), D=512, H=64, H_I=16, d_I=128, topk=256,
+                       pool_blocks=64, modes=("full", "reuse", "reuse", "reindex", "reuse"))
+    a = DeviceWorkload(W, use_stash=True)
+    b = DeviceWorkload(W, use_stash=False)
+    assert a.stash is not None and b.stash is None
+    a.run_step()
+    b.run_step()
+    torch.cuda.synchronize()
+    for li in range(len(W.modes)):
+        assert torch.equal(a.out[li], b.out[li]), li
+        assert torch.equal(a.lse[li], b.lse[li]), li
