@@ -140,20 +140,32 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   if (kGather) {
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = 0;
     __syncthreads();
-    const int64_t n = (int64_t)a.num_q * a.pool_blocks;
+    // (num_q <= 4096 and pool_blocks <= 8192 keep every index below 2^25: 32-bit math)
+    const int n = a.num_q * a.pool_blocks;
     const int32_t* pl = a.pool + (int64_t)a.q0 * a.pool_blocks;
-    for (int64_t b0 = 0; b0 < n; b0 += 16 * kScoreThreads) {    // 16 loads in flight
+    for (int b0 = 0; b0 < n; b0 += 16 * kScoreThreads) {    // 16 loads in flight
       int32_t v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int64_t i = b0 + j * kScoreThreads + tid;
+        const int i = b0 + j * kScoreThreads + tid;
         v[j] = i < n ? __ldg(pl + i) : -1;
       }
+      // count valid entries per row in a register; one shared atomic per row change
+      int cur_row = -1;
+      uint32_t cnt = 0;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int64_t i = b0 + j * kScoreThreads + tid;
-        if (v[j] >= 0) atomicAdd(&rowp[i / a.pool_blocks + 1], 1u);   // valid pool entries
+        const int i = b0 + j * kScoreThreads + tid;
+        if (i >= n) break;
+        const int row = i / a.pool_blocks;
+        if (row != cur_row) {
+          if (cnt) atomicAdd(&rowp[cur_row + 1], cnt);
+          cur_row = row;
+          cnt = 0;
+        }
+        cnt += v[j] >= 0;
       }
+      if (cnt) atomicAdd(&rowp[cur_row + 1], cnt);
     }
     __syncthreads();
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = (rowp[i + 1] + 15) / 16;
@@ -169,10 +181,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     fence_barrier_init();
   }
   // padding rows of the B operand (heads >= H_I) must read as zero; TMA never writes them
-  for (int s = 0; s < S; ++s) {
-    uint8_t* b = base + (size_t)s * stage_bytes + a_bytes;
-    for (uint32_t i = tid * 16; i < (uint32_t)halves * b_half; i += kScoreThreads * 16)
-      *reinterpret_cast<uint4*>(b + i) = make_uint4(0, 0, 0, 0);
+  if (a.H_I < a.n_pad) {
+    const uint32_t pad = (uint32_t)(a.n_pad - a.H_I) * 128;
+    for (int s = 0; s < S; ++s) {
+      uint8_t* b = base + (size_t)s * stage_bytes + a_bytes;
+      for (uint32_t i = tid * 16; i < (uint32_t)halves * pad; i += kScoreThreads * 16) {
+        const uint32_t h = i / pad, o = i % pad;
+        *reinterpret_cast<uint4*>(b + h * b_half + (uint32_t)a.H_I * 128 + o) = make_uint4(0, 0, 0, 0);
+      }
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -619,7 +636,7 @@ __device__ void final_select(const SelProblem& p, int r, const Top& tp, const Sr
 
 constexpr int kStageCap = 12288;       // candidates staged in shared memory (96 KB)
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a) {
   extern __shared__ uint4 stage_raw[];      // chunk keys, later [kStageCap] keys + positions
   uint32_t* stage_buf = reinterpret_cast<uint32_t*>(stage_raw);
   __shared__ uint32_t red[kSelThreads / 32];
@@ -663,12 +680,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
     // append this chunk's candidates in position order: warp w owns a contiguous eighth
     const int sub = kSelChunk / (kSelThreads / 32);
     const int w_lo = wid * sub, w_hi = min(hi - lo, w_lo + sub);   // chunk-relative
-    auto is_cand = [&](int i) {
-      const uint32_t k = stage_buf[i];
-      return i < w_hi && k != 0u && (k >> 21) >= tp.b1;
-    };
+    // this warp's keys in registers (key k of lane l: chunk position w_lo + 32 k + l)
+    constexpr int kPerLane = kSelChunk / kSelThreads;       // 32
+    uint32_t kk[kPerLane];
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) {
+      const int i = w_lo + 32 * k + lane;
+      const uint32_t key = i < w_hi ? stage_buf[i] : 0u;
+      kk[k] = (key != 0u && (key >> 21) >= tp.b1) ? key : 0u;   // 0: not a candidate
+    }
     uint32_t cnt = 0;
-    for (int b0 = w_lo; b0 < w_hi; b0 += 32) cnt += __popc(__ballot_sync(0xffffffffu, is_cand(b0 + lane)));
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) cnt += __popc(__ballot_sync(0xffffffffu, kk[k] != 0u));
     if (lane == 0) wcnt[wid] = cnt;
     __syncthreads();
     if (tid == 0) {
@@ -682,14 +705,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
     uint32_t o = s_base + wcnt[wid];
     uint32_t* cand = p.cand + (int64_t)r * p.cand_cap;
     uint32_t* cand_key = p.cand_key + (int64_t)r * p.cand_cap;
-    for (int b0 = w_lo; b0 < w_hi; b0 += 32) {
-      const int i = b0 + lane;
-      const bool pr = is_cand(i);
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) {
+      const bool pr = kk[k] != 0u;
       const uint32_t m = __ballot_sync(0xffffffffu, pr);
       if (pr) {
-        const uint32_t at = o + __popc(m & lanemask_lt());
-        cand[at] = (uint32_t)(lo + i);
-        cand_key[at] = stage_buf[i];
+        const uint32_t at = o + __popc(m & lt);
+        cand[at] = (uint32_t)(lo + w_lo + 32 * k + lane);
+        cand_key[at] = kk[k];
       }
       o += __popc(m);
     }
