@@ -5,24 +5,30 @@
 // and window KV; Reuse layers attend with the latest indices) and "FP4 KV 与部署层的几个改动"
 // (E2M1 values with one E4M3 scale per 16 channels).
 //
-// One CTA handles a range of 128-key tiles of one query.  The key slots of a query are
-// [indices[q][0..topk) ; window positions t-W+1 .. t].  Per tile:
-//   gather   all 8 warps load the tile's rows -- FP4 rows are dequantised in registers to
-//            bf16 (exact: a 2-bit-mantissa code times a 4-bit-mantissa scale), window rows
-//            are copied with cp.async -- into a 128-byte-swizzled [128 keys x D] tile;
+// One CTA handles a range of 128-key tiles of one query for one group of 16 or 32 heads
+// (the key slots of a query are [indices[q][0..topk) ; window positions t-W+1 .. t]).
+// Per tile:
+//   stage    the selected rows' FP4 codes and scales are copied with cp.async (row-
+//            contiguous, 16-byte pieces) into a staging area -- or, in a Reuse layer with
+//            a stash, come back as one bulk copy of the stage image that the group's
+//            Full / Reindex call stored; window rows go by cp.async straight into the tile;
+//   dequant  all 8 warps decode the staged rows to bf16 (exact: a 2-bit-mantissa code times
+//            a 4-bit-mantissa scale) into a 128-byte-swizzled [128 keys x D] tile;
 //   S^T      one thread issues tcgen05.mma: S^T[key, head] = KV[key, :] . Q[head, :]
-//            (M = 128 keys, N = heads, K = D; Q arrives once by TMA);
-//   softmax  warps 0-3 read S^T from TMEM (one key per thread), form per-head maxima and
-//            sums with warp reduce-scatters, keep a lazily rescaled running max per head,
-//            and write P (bf16) as [key][head] rows -- an MN-major operand;
+//            (M = 128 keys, N = the CTA's heads, K = D; Q arrives once by TMA);
+//   softmax  all 8 warps read S^T from TMEM (one key per thread, half the heads per warp),
+//            form per-head maxima and sums with warp reduce-scatters, keep a lazily
+//            rescaled running max per head, and write P (bf16) as [head][key] rows;
 //   O^T      tcgen05.mma: O^T[d, head] += V^T[d, key] . P^T[key, head], reading the same
-//            swizzled KV tile as an MN-major operand (M = 128 dims per slab, N = heads).
-// The last tile's O^T is normalised and written; when a query is split over several CTAs
-// they write (m, l, O) partials that a small kernel merges by log-sum-exp.
+//            swizzled KV tile as an MN-major operand (M = 128 dims per slab).
+// The last tile's O^T is normalised and written straight from TMEM; when a query is split
+// over several CTAs they write (m, l, O) partials that a small kernel merges by
+// log-sum-exp.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -33,6 +39,7 @@ constexpr int kThreads = 256;                // 8 warps
 constexpr int kTile = 128;                   // keys per tile (MMA M)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;         // rescale O only when a max grows by > 2^8
+constexpr int kScaleStride = 48;             // bytes per staged scale row (16-aligned)
 
 struct AttnArgs {
   int num_q;
@@ -50,9 +57,10 @@ struct AttnArgs {
   const int64_t* q_pos;
   int window;
   int mode;                                  // csa2_mode_t
-  uint8_t* stash;                            // [num_q][n_idx_tiles][tile bytes] or null
+  uint8_t* stash;                            // [num_q][n_idx_tiles][stage bytes] or null
   int n_idx_tiles;                           // tiles holding index slots: ceil(topk / 128)
-  int H;                                     // real heads (<= kN); the rest are padding
+  int H;                                     // real heads
+  int hsplit;                                // head groups (CTAs) per query and split
   float scale_log2;                          // softmax_scale * log2(e)
   int n_tiles;                               // tiles of the slot list
   int nsplit, tiles_per_split;
@@ -63,19 +71,38 @@ struct AttnArgs {
   int* status;
 };
 
-constexpr int kN = 64;                       // MMA N: heads, padded to 64
+// Shared-memory geometry of one CTA (offsets from a 1024-byte aligned base).
+template <int D, int HN>
+struct Geo {
+  static constexpr int kChunks = D / 64;               // 64-element (128-byte) column chunks
+  static constexpr int kSlabs = D / 128;               // O^T slabs of 128 dims (MMA M)
+  static constexpr uint32_t kQChunk = HN * 128;        // Q chunk: [HN rows][128 B]
+  static constexpr uint32_t kKVChunk = kTile * 128;    // KV chunk: [128 keys][128 B]
+  static constexpr uint32_t kPChunk = HN * 128;        // P chunk: [HN heads][64 keys]
+  static constexpr uint32_t kCodeStride = D / 2 + 16;  // staged code row (padded: no bank conflicts)
+  static constexpr uint32_t kStageCodes = kTile * kCodeStride;
+  static constexpr uint32_t kStageBytes = kStageCodes + kTile * kScaleStride;
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = (kChunks * kQChunk + 1023) / 1024 * 1024;
+  static constexpr uint32_t kOffP = kOffKV + kChunks * kKVChunk;
+  static constexpr uint32_t kOffStage = kOffP + (2 * kPChunk + 1023) / 1024 * 1024;
+  static constexpr uint32_t kSmem = 1024 + kOffStage + kStageBytes;
+  static constexpr uint32_t kTmemCols = (HN + kSlabs * HN) <= 128 ? 128 : 256;
+  static_assert(kStageBytes % 16 == 0 && D / 16 <= kScaleStride, "stage layout");
+};
 
-template <int H>
+template <int HN>
 struct AttnSmem {
   uint64_t bar_q, bar_s, bar_o, bar_kv;
   uint32_t tmem_base;
   int abort;
   int rescale;
-  float m_ref[H];
-  float l_acc[H];
-  float alpha[H];
-  float red[4][H];
-  int valid[kTile];
+  float m_ref[HN];
+  float l_acc[HN];
+  float alpha[HN];
+  float red[4][HN];
+  int kind[kTile];                           // 0 invalid, 1 FP4 row, 2 window row
+  int64_t src[kTile];                        // cache row (kind 1) or window row (kind 2)
 };
 
 // non-negative e4m3 scale byte -> value (bias 7; exponent field 0 is subnormal m * 2^-9)
@@ -143,38 +170,53 @@ __device__ __forceinline__ void reduce_scatter_step(float* v, int lane) {
   }
 }
 
-template <int D>
+// Per-head reduction of v[0..N) over the 32 lanes (keys) of a warp: afterwards v[0] of
+// lane l is the warp-wide result for head l mod N.
+template <int N, bool kMax>
+__device__ __forceinline__ void warp_reduce_heads(float* v, int lane) {
+  reduce_scatter_step<N, N / 2, kMax>(v, lane);
+#pragma unroll
+  for (int b = N; b < 32; b <<= 1) {
+    const float y = __shfl_xor_sync(0xffffffffu, v[0], b);
+    v[0] = kMax ? fmaxf(v[0], y) : v[0] + y;
+  }
+}
+
+template <int D, int HN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
-  constexpr int H = kN;
-  constexpr int kChunks = D / 64;            // 64-element (128-byte) column chunks
-  constexpr int kSlabs = D / 128;            // O^T slabs of 128 dims (MMA M)
-  constexpr uint32_t kQChunk = H * 128;      // bytes of one Q chunk ([H rows][128 B])
-  constexpr uint32_t kQBytes = kChunks * kQChunk;
-  constexpr uint32_t kKVChunk = kTile * 128;  // 16 KB
-  constexpr uint32_t kTmemCols = (H + kSlabs * H) <= 128 ? 128 : ((H + kSlabs * H) <= 256 ? 256 : 512);
-  static_assert(D % 128 == 0 && D <= 512, "shape");
+  using G = Geo<D, HN>;
+  constexpr int kChunks = G::kChunks, kSlabs = G::kSlabs;
+  constexpr int HW = HN / 2;                 // heads per warp in softmax and epilogue
+  constexpr int kParts = D / 32;             // 16-byte code pieces (32 values) of a row
+  constexpr int kRowsPerIter = kThreads / kParts;
+  constexpr int kIters = kTile / kRowsPerIter;
+  constexpr uint32_t kKVChunk = G::kKVChunk;
   const int Hr = a.H;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ AttnSmem<H> ss;
+  __shared__ AttnSmem<HN> ss;
   // 1024-byte aligned base, derived from the shared array itself so that the compiler keeps
   // the shared address space (and knows these buffers do not alias `ss`)
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sQ = base;
-  uint8_t* sKV = sQ + ((kQBytes + 1023) / 1024) * 1024;
-  uint8_t* sP = sKV + kChunks * kKVChunk;
+  uint8_t* sQ = base + G::kOffQ;
+  uint8_t* sKV = base + G::kOffKV;
+  uint8_t* sP = base + G::kOffP;
+  uint8_t* sStage = base + G::kOffStage;
+  uint8_t* sScale = sStage + G::kStageCodes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-  const int hh = warp >> 2;                  // head half (softmax / epilogue columns)
-  const int split = blockIdx.x, q = blockIdx.y;
+  const int h0 = (warp >> 2) * HW;           // this warp's heads [h0, h0 + HW) of the group
+  const int hg = blockIdx.x % a.hsplit, split = blockIdx.x / a.hsplit, q = blockIdx.y;
+  const int h_lo = hg * HN;                  // first head of the CTA's group
   const int seq = q / a.q_per_seq;
   const int t_begin = split * a.tiles_per_split;
   const int t_end = min(a.n_tiles, t_begin + a.tiles_per_split);
   volatile int* abort = &ss.abort;
 
-  // Q goes out first: barrier init, then its TMA, by one thread
+  // set-up that reads no global memory (it overlaps the previous kernel's tail)
+  pdl_trigger();
   if (tid == 0) {
     mbar_init(&ss.bar_q, 1);
     mbar_init(&ss.bar_s, 1);
@@ -183,9 +225,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     ss.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
-    mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * Hr * 128);
-    for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunk, &tm_q, c * 64, q * Hr, &ss.bar_q);
   }
+  if (tid < HN) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
+  if (warp == 0) { tmem_alloc(&ss.tmem_base, G::kTmemCols); tmem_relinquish(); }
+  pdl_wait();
+  // Q of the group first, by one thread (heads >= H read as zero: the box runs past the map)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * G::kQChunk);
+    for (int c = 0; c < kChunks; ++c)
+      tma_load_3d(sQ + c * G::kQChunk, &tm_q, c * 64, h_lo, q, &ss.bar_q);
+  }
+  // index of row `tid` of a tile (threads < 128), fetched one tile ahead
+  int32_t my_idx = 0;
+  auto fetch_idx = [&](int t) {
+    const int slot = t * kTile + tid;
+    if (tid < kTile && slot < a.topk) my_idx = __ldg(a.indices + (int64_t)q * a.topk + slot);
+  };
+  if (t_begin < t_end) fetch_idx(t_begin);
 
   const int64_t row0 = a.seq_start[seq];
   const int slen = a.seq_len[seq];
@@ -194,67 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_win = (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0);
   const int64_t wrow0 = a.swa_start[seq] + w0;
 
-  // gather geometry: kParts threads per row, each covering 32 columns (4 units of 8 bf16)
-  constexpr int kParts = D / 32;
-  constexpr int kRowsPerIter = kThreads / kParts;
-  constexpr int kIters = kTile / kRowsPerIter;
-  // consecutive threads take consecutive rows: the 8 threads of a quarter warp then store
-  // to 8 different rows, whose 128-byte swizzle puts their 16-byte units in 8 bank groups
-  const int rsub = tid % kRowsPerIter;
-  const int part = tid / kRowsPerIter;
-  int kind[kIters];                          // 0 invalid, 1 FP4 row, 2 window row
-  int32_t gidx[kIters];                      // FP4: sequence position; window: offset in window
-  // Phase 1 of a tile's gather: slot -> source (the index load is only issued here).
-  auto issue_slots = [&](int t) {
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int slot = t * kTile + it * kRowsPerIter + rsub;
-      kind[it] = 0;
-      gidx[it] = 0;
-      if (slot < a.topk) {
-        gidx[it] = __ldg(a.indices + (int64_t)q * a.topk + slot);
-        kind[it] = 1;
-      } else if (slot - a.topk < n_win) {
-        gidx[it] = slot - a.topk;
-        kind[it] = 2;
-      }
-    }
-  };
-  if (t_begin < t_end) issue_slots(t_begin);
-
-  if (tid < H) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
-  if (Hr < H) {  // rows of padding heads must read as zero; TMA writes rows < Hr only
-    const uint32_t pad = (uint32_t)(H - Hr) * 128;
-    for (uint32_t i = tid * 16; i < kChunks * pad; i += kThreads * 16) {
-      const uint32_t c = i / pad, o = i % pad;
-      *reinterpret_cast<uint4*>(sQ + c * kQChunk + (uint32_t)Hr * 128 + o) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-  }
-  if (warp == 0) { tmem_alloc(&ss.tmem_base, kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem_base;
-  const uint32_t tS = tmem;                  // S^T: columns [0, H)
-  const uint32_t tO = tmem + H;              // O^T slab j: columns [H + jH, H + (j+1)H)
+  const uint32_t tS = tmem;                  // S^T: columns [0, HN)
+  const uint32_t tO = tmem + HN;             // O^T slab j: columns [HN + j HN, HN + (j+1) HN)
   const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
-  const uint32_t idesc_s = idesc_bf16(kTile, H);
-  const uint32_t idesc_o = idesc_bf16(kTile, H, true, true);
+  const uint32_t idesc_s = idesc_bf16(kTile, HN);                  // KV, Q both K-major
+  const uint32_t idesc_o = idesc_bf16(kTile, HN, true, false);     // V^T MN-major, P K-major
   uint32_t ph_s = 0, ph_o = 0, ph_kv = 0;
   bool q_ready = false, o_init = false, o_pending = false, store_pending = false;
-  constexpr uint32_t kTileBytes = kChunks * kKVChunk;
 
   for (int t = t_begin; t < t_end; ++t) {
-    // Reuse with a stash: this tile's selected rows come back as the bf16 tile a Full /
-    // Reindex call stored; Full / Reindex with a stash store their tile after the gather.
+    // Reuse with a stash: the tile's selected rows come back as the stage image that the
+    // Full / Reindex call (head group 0) stored after its gather.
     const bool stash_tile = a.stash != nullptr && t < a.n_idx_tiles;
     const bool from_stash = stash_tile && a.mode == CSA2_MODE_REUSE;
-    const bool to_stash = stash_tile && a.mode != CSA2_MODE_REUSE;
-    uint8_t* stile = stash_tile ? a.stash + ((int64_t)q * a.n_idx_tiles + t) * kTileBytes : nullptr;
-    if (t != t_begin) issue_slots(t);        // in flight while the previous O^T finishes
-    // the previous tile's O^T MMA must be done before its KV / P buffers are rewritten
+    const bool to_stash = stash_tile && a.mode != CSA2_MODE_REUSE && hg == 0;
+    uint8_t* stile = stash_tile ? a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStageBytes : nullptr;
+    // the previous tile's O^T MMA and stash store must be done before its buffers are rewritten
     if (store_pending && tid == 0) bulk_wait_read();
     if (o_pending) {
       const bool ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status);
@@ -266,109 +282,144 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
     }
     store_pending = false;
-    if (from_stash) {
-      if (tid == 0) {
-        mbar_arrive_expect_tx(&ss.bar_kv, kTileBytes);
-        for (int c = 0; c < kChunks; ++c)
-          bulk_g2s(sKV + c * kKVChunk, stile + c * kKVChunk, kKVChunk, &ss.bar_kv);
-      }
-      const bool ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
-      ph_kv ^= 1;
-      if (__syncthreads_or(!ok)) break;
+    if (from_stash && tid == 0) {            // needs no index: goes out first
+      mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
+      bulk_g2s(sStage, stile, G::kStageBytes, &ss.bar_kv);
     }
-    // ------------------------------ gather ------------------------------
-    // Phase 2: the rows -- FP4 codes + scales into registers, window rows by cp.async
-    // straight to shared memory; phase 3: dequantise (LUT + exact bf16 multiply) and store
-    // into the 128-byte-swizzled [128 keys x D] tile.
-    uint4 cw[kIters];
-    uint32_t sc[kIters];
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int r = it * kRowsPerIter + rsub;
-      uint8_t* row_smem = sKV + r * 128;
-      if (kind[it] == 1) {
-        const int p = gidx[it];
+    // ------------------------- slots -> sources (one thread per row) -------------------------
+    if (tid < kTile) {
+      const int slot = t * kTile + tid;
+      int kind = 0;
+      int64_t src = 0;
+      if (slot < a.topk) {
+        const int p = my_idx;
         if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
-          if (from_stash) {
-            kind[it] = 3;                          // row already in the tile (from the stash)
-          } else {
-            const int64_t grow = row0 + p;
-            cw[it] = __ldg(reinterpret_cast<const uint4*>(a.codes + grow * (D / 2) + part * 16));
-            sc[it] = __ldg(reinterpret_cast<const uint16_t*>(a.scales + grow * (D / 16) + part * 2));
-          }
-        } else {
-          if (p >= slen || p < -1) report(a.status, CSA2_ERR_INVALID_ARG);
-          else if (p >= 0) report(a.status, CSA2_ERR_CAPACITY);
-          kind[it] = 0;
+          kind = 1;
+          src = row0 + p;
+        } else if (p >= slen || p < -1) {
+          report(a.status, CSA2_ERR_INVALID_ARG);
+        } else if (p >= 0) {
+          report(a.status, CSA2_ERR_CAPACITY);
         }
-      } else if (kind[it] == 2) {
-        const int64_t grow = wrow0 + gidx[it];
+      } else if (slot - a.topk < n_win) {
+        const int64_t grow = wrow0 + (slot - a.topk);
         if (grow >= 0 && grow < a.swa_rows) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int u = 4 * part + i;
-            cp_async16(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4),
-                       a.swa + grow * D + u * 8);
-          }
+          kind = 2;
+          src = grow;
         } else {
           report(a.status, CSA2_ERR_CAPACITY);
-          kind[it] = 0;
         }
       }
+      ss.kind[tid] = kind;
+      ss.src[tid] = src;
     }
+    __syncthreads();
+    if (t + 1 < t_end) fetch_idx(t + 1);
+    // ------------------------- loads (a row's threads are contiguous) -------------------------
+    {
+      const int lp = tid % kParts;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int r = it * kRowsPerIter + rsub;
-      uint8_t* row_smem = sKV + r * 128;
-      if (part == 0) ss.valid[r] = kind[it] != 0;
-      if (kind[it] == 1) {
-        const float s0 = e4m3_val(sc[it] & 0xFFu), s1 = e4m3_val((sc[it] >> 8) & 0xFFu);
-        const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
-        const uint32_t w4[4] = {cw[it].x, cw[it].y, cw[it].z, cw[it].w};
+      for (int it = 0; it < kIters; ++it) {
+        const int r = it * kRowsPerIter + tid / kParts;
+        const int kind = ss.kind[r];
+        if (kind == 1 && !from_stash) {
+          const int64_t grow = ss.src[r];
+          cp_async16(sStage + r * G::kCodeStride + lp * 16, a.codes + grow * (D / 2) + lp * 16);
+          if constexpr (D / 16 >= 16) {
+            if (lp * 16 < D / 16) cp_async16(sScale + r * kScaleStride + lp * 16, a.scales + grow * (D / 16) + lp * 16);
+          } else {
+            if (lp == 0) cp_async8(sScale + r * kScaleStride, a.scales + grow * (D / 16));
+          }
+        } else if (kind == 2) {
+          const uint16_t* src = a.swa + ss.src[r] * D;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {              // unit i: 8 values of word w4[i]
-          const uint32_t s2 = i < 2 ? s02 : s12;
-          uint4 o;
-          uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-          e2m1x8_to_bf16(w4[i], ow);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ow[k], s2);
-          const int u = 4 * part + i;
-          *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
-        }
-      } else if (kind[it] == 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int u = 4 * part + i;
-          *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) =
-              make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) {
+            const int u = 4 * lp + i;
+            cp_async16(sKV + (u >> 3) * kKVChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4), src + u * 8);
+          }
+        } else if (kind == 0 && to_stash && t * kTile + r < a.topk) {
+          // an index slot without a row is stored as zero codes and scales
+          *reinterpret_cast<uint4*>(sStage + r * G::kCodeStride + lp * 16) = make_uint4(0, 0, 0, 0);
+          if (lp * 16 < D / 16) {
+            if constexpr (D / 16 >= 16)
+              *reinterpret_cast<uint4*>(sScale + r * kScaleStride + lp * 16) = make_uint4(0, 0, 0, 0);
+            else
+              *reinterpret_cast<uint2*>(sScale + r * kScaleStride) = make_uint2(0, 0);
+          }
         }
       }
     }
     cp_async_wait_all();
-    fence_proxy_async_smem();
-    const int any = __syncthreads_or(ss.valid[tid & (kTile - 1)]);
-    if (to_stash) {                            // keep the dequantised tile for Reuse layers
+    bool ok = true;
+    if (from_stash) {
+      ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
+      ph_kv ^= 1;
+    }
+    if (to_stash) fence_proxy_async_smem();  // staged rows -> the bulk store below
+    if (__syncthreads_or(!ok)) break;
+    if (to_stash) {
       if (tid == 0) {
-        for (int c = 0; c < kChunks; ++c) bulk_s2g(stile + c * kKVChunk, sKV + c * kKVChunk, kKVChunk);
+        bulk_s2g(stile, sStage, G::kStageBytes);
         bulk_commit();
       }
-      store_pending = true;                    // uniform: every thread takes the same branches
+      store_pending = true;                  // uniform: every thread takes the same branches
     }
+    // ------------------------- dequantise into the swizzled tile -------------------------
+    // consecutive threads take consecutive rows: the 8 threads of a quarter warp then store
+    // to 8 different rows, whose 128-byte swizzle puts their 16-byte units in 8 bank groups
+    {
+      const int rsub = tid % kRowsPerIter;
+      const int part = tid / kRowsPerIter;
+#pragma unroll
+      for (int it = 0; it < kIters; ++it) {
+        const int r = it * kRowsPerIter + rsub;
+        const int kind = ss.kind[r];
+        uint8_t* row_smem = sKV + r * 128;
+        // a stash holds zero codes for index slots without a row
+        const bool dec = from_stash ? (t * kTile + r < a.topk) : (kind == 1);
+        if (dec) {
+          const uint4 cw = *reinterpret_cast<const uint4*>(sStage + r * G::kCodeStride + part * 16);
+          const uint32_t sc = *reinterpret_cast<const uint16_t*>(sScale + r * kScaleStride + part * 2);
+          const float s0 = e4m3_val(sc & 0xFFu), s1 = e4m3_val((sc >> 8) & 0xFFu);
+          const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
+          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {              // unit i: 8 values of word w4[i]
+            const uint32_t s2 = i < 2 ? s02 : s12;
+            uint4 o;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+            e2m1x8_to_bf16(w4[i], ow);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ow[k], s2);
+            const int u = 4 * part + i;
+            *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
+          }
+        } else if (kind == 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int u = 4 * part + i;
+            *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    const int any = __syncthreads_or(tid < kTile && ss.kind[tid] != 0);
     if (!any) continue;
 
     // ------------------------------ S^T = KV . Q^T ------------------------------
     if (tid == 0) {
-      bool ok = true;
-      if (!q_ready) { ok = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = ok; }
-      if (ok) {
+      bool okq = true;
+      if (!q_ready) { okq = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = okq; }
+      if (okq) {
         tc_fence_after();
         const uint64_t kv_desc_k = sdesc_sw128(smem_u32(sKV), 16, 1024);   // KV as K-major A
         const uint64_t q_desc_k = sdesc_sw128(smem_u32(sQ), 16, 1024);     // Q as K-major B
 #pragma unroll 4
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * kKVChunk + (k & 3) * 32;
-          const uint32_t qoff = (uint32_t)(k >> 2) * kQChunk + (k & 3) * 32;
+          const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunk + (k & 3) * 32;
           umma_bf16(tS, kv_desc_k + (off >> 4), q_desc_k + (qoff >> 4), idesc_s, k > 0 ? 1u : 0u);
         }
         umma_commit(&ss.bar_s);
@@ -376,29 +427,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ------------------------------ softmax (all 8 warps) ------------------------------
-    // warp w: keys of TMEM lane quadrant (w & 3), heads [32 * (w >> 2), +32)
+    // warp w: keys of TMEM lane quadrant (w & 3), heads [h0, h0 + HW)
     const int r = quad * 32 + lane;               // key row = TMEM lane
-    const int h0 = hh * 32;
-    float v[32];
-    bool ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
+    float v[HW];
+    ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
     ok = __syncthreads_and(ok);
     ph_s ^= 1;
     if (!ok) break;
     tc_fence_after();
-    tmem_ld32(tS + lane_base + h0, tS + lane_base + h0 + 16, v);
+    tmem_ldn<HW>(tS + lane_base + h0, v);
     {
-      const bool valid = ss.valid[r] != 0;
+      const bool valid = ss.kind[r] != 0;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
-      float red[32];
+      for (int h = 0; h < HW; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
+      float red[HW];
 #pragma unroll
-      for (int h = 0; h < 32; ++h) red[h] = v[h];
-      reduce_scatter_step<32, 16, true>(red, lane);     // lane holds head h0 + lane
-      ss.red[quad][h0 + lane] = red[0];
+      for (int h = 0; h < HW; ++h) red[h] = v[h];
+      warp_reduce_heads<HW, true>(red, lane);     // lane holds head h0 + lane % HW
+      if (lane < HW) ss.red[quad][h0 + lane] = red[0];
     }
     if (tid == 0) ss.rescale = 0;
     __syncthreads();
-    if (tid < H) {
+    if (tid < HN) {
       const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
       ss.alpha[tid] = mt;                          // stash the tile max
       if (mt > ss.m_ref[tid] + kRescaleLog2) ss.rescale = 1;
@@ -406,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (ss.rescale) {
       // move every head's reference max up to its running max; O and l scale by alpha
-      if (tid < H) {
+      if (tid < HN) {
         const float mo = ss.m_ref[tid];
         const float mn = fmaxf(mo, ss.alpha[tid]);
         const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
@@ -416,61 +466,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       if (o_init) {
-        float al[32];
+        float al[HW];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) al[i] = ss.alpha[h0 + i];
+        for (int i = 0; i < HW; ++i) al[i] = ss.alpha[h0 + i];
 #pragma unroll 1
         for (int j = 0; j < kSlabs; ++j) {
-          float o[32];
-          const uint32_t ta = tO + lane_base + j * H + h0;
-          tmem_ld32(ta, ta + 16, o);
+          float o[HW];
+          const uint32_t ta = tO + lane_base + j * HN + h0;
+          tmem_ldn<HW>(ta, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= al[i];
-          tmem_st16(ta, o);
-          tmem_st16(ta + 16, o + 16);
+          for (int i = 0; i < HW; ++i) o[i] *= al[i];
+          tmem_stn<HW>(ta, o);
         }
         tmem_wait_st();
       }
     }
     {
-      // p = 2^(s - m_ref), rounded to bf16; P row r = [heads] (the MN-major B operand)
-      // (v is overwritten with the bf16-rounded p for the per-head sums)
+      // p = 2^(s - m_ref), rounded to bf16, written as P[head][key] (a K-major operand:
+      // two 64-key chunks of [HN rows x 128 B], 128-byte swizzle); v becomes the rounded p
+      uint8_t* prow = sP + (r >> 6) * G::kPChunk;
+      const uint32_t unit = (uint32_t)(r & 63) >> 3, byte = (uint32_t)(r & 7) * 2;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint4 pk;
-        uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int h = 8 * u + 2 * k;
-          const float p0 = fast_exp2(v[h] - ss.m_ref[h0 + h]);
-          const float p1 = fast_exp2(v[h + 1] - ss.m_ref[h0 + h + 1]);
-          pw[k] = pack_bf16(p0, p1);
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[k]));
-          v[h] = f.x;
-          v[h + 1] = f.y;
-        }
-        const int unit = 4 * hh + u;
-        *reinterpret_cast<uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
+      for (int i = 0; i < HW; ++i) {
+        const int h = h0 + i;
+        const __nv_bfloat16 pb = __float2bfloat16_rn(fast_exp2(v[i] - ss.m_ref[h]));
+        v[i] = __bfloat162float(pb);
+        *reinterpret_cast<__nv_bfloat16*>(prow + h * 128 + ((unit ^ (h & 7)) << 4) + byte) = pb;
       }
-      reduce_scatter_step<32, 16, false>(v, lane);
-      ss.red[quad][h0 + lane] = v[0];
+      warp_reduce_heads<HW, false>(v, lane);
+      if (lane < HW) ss.red[quad][h0 + lane] = v[0];
       fence_proxy_async_smem();
       tc_fence_before();
     }
     __syncthreads();
-    if (tid < H) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
+    if (tid < HN) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
     // ------------------------------ O^T += V^T . P^T ------------------------------
     if (tid == 0) {
       tc_fence_after();
       const uint64_t kv_desc_mn = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);  // V^T, MN-major A
-      const uint64_t p_desc_mn = sdesc_sw128(smem_u32(sP), 8192, 1024);        // P^T, MN-major B
+      const uint64_t p_desc_k = sdesc_sw128(smem_u32(sP), 16, 1024);           // P, K-major B
 #pragma unroll 1
       for (int j = 0; j < kSlabs; ++j) {
 #pragma unroll 4
         for (int k = 0; k < kTile / 16; ++k) {
           const uint32_t off = (uint32_t)(2 * j) * kKVChunk + k * 2048;
-          umma_bf16(tO + j * H, kv_desc_mn + (off >> 4), p_desc_mn + ((uint32_t)(k * 2048) >> 4),
-                    idesc_o, (o_init || k > 0) ? 1u : 0u);
+          const uint32_t poff = (uint32_t)(k >> 2) * G::kPChunk + (k & 3) * 32;
+          umma_bf16(tO + j * HN, kv_desc_mn + (off >> 4), p_desc_k + (poff >> 4), idesc_o,
+                    (o_init || k > 0) ? 1u : 0u);
         }
       }
       umma_commit(&ss.bar_o);
@@ -486,169 +528,99 @@ __global__ void __launch_bounds__(kThreads, 1)
   done_ok = __syncthreads_and(done_ok);
   tc_fence_after();
   const bool partial = a.nsplit > 1;
-  if (partial) {
-    // Split query: write this CTA's unnormalised O (relative to m_ref) as [D][Hr] rows,
-    // straight from TMEM (16-byte stores of 32 heads per thread), plus (m, l) per head.
-    if (done_ok) {
-      float* po = a.part_o + ((int64_t)q * a.nsplit + split) * D * Hr;
-      const int hbase = hh * 32;
-#pragma unroll 1
-      for (int j = 0; j < kSlabs; ++j) {
-        const int d = j * 128 + quad * 32 + lane;
-        float o[32];
-        if (o_init) {
-          const uint32_t ta = tO + lane_base + j * H + hbase;
-          tmem_ld32(ta, ta + 16, o);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.0f;
-        }
-        float* row = po + (int64_t)d * Hr + hbase;
-        if (hbase + 32 <= Hr && (Hr & 3) == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(row + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (hbase + i < Hr) row[i] = o[i];
-        }
-      }
-      if (tid < Hr) {
-        const float m = ss.m_ref[tid], l = ss.l_acc[tid];
-        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + tid) * 2;
-        ml[0] = (o_init && l > 0.0f) ? m : -INFINITY;
-        ml[1] = o_init ? l : 0.0f;
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
-    }
-    return;
-  }
-  if (tid < H) {  // reciprocal of l for the normalised (unsplit) output
-    const float l = ss.l_acc[tid];
-    ss.alpha[tid] = (!partial && l > 0.0f) ? 1.0f / l : 1.0f;
-  }
-  __syncthreads();
-  // The KV tile is free once the last O^T MMA has completed: stage O there as [head][D]
-  // fp32, then copy it out with 16-byte stores.
-  float* so = reinterpret_cast<float*>(sKV);        // [Hr][D] (Hr * D * 4 <= 128 KB)
   if (done_ok) {
-    const int hbase = hh * 32;
-    float oscale[32];
+    // Straight from TMEM: a thread holds one dim of HW heads, so a warp stores one full
+    // 128-byte line per head.  Unsplit: out = O / l.  Split: the unnormalised O (relative
+    // to m_ref) as [H][D] rows of this split, plus (m, l) per head.
+    float* dst = partial ? a.part_o + ((int64_t)q * a.nsplit + split) * Hr * D
+                         : a.out + (int64_t)q * Hr * D;
+    float osc[HW];
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      oscale[i] = (o_init && ss.l_acc[hbase + i] > 0.0f) ? ss.alpha[hbase + i] : 0.0f;
+    for (int i = 0; i < HW; ++i) {
+      const float l = ss.l_acc[h0 + i];
+      osc[i] = !o_init ? 0.0f : (partial ? 1.0f : (l > 0.0f ? 1.0f / l : 0.0f));
+    }
 #pragma unroll 1
     for (int j = 0; j < kSlabs; ++j) {
       const int d = j * 128 + quad * 32 + lane;
-      float o[32];
+      float o[HW];
       if (o_init) {
-        const uint32_t ta = tO + lane_base + j * H + hbase;
-        tmem_ld32(ta, ta + 16, o);
+        tmem_ldn<HW>(tO + lane_base + j * HN + h0, o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < HW; ++i) o[i] = 0.0f;
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int h = hbase + i;
-        if (h < Hr) so[h * D + d] = o_init ? o[i] * oscale[i] : 0.0f;
+      for (int i = 0; i < HW; ++i) {
+        const int h = h_lo + h0 + i;
+        if (h < Hr) dst[h * D + d] = o[i] * osc[i];
       }
     }
-    if (tid < Hr) {
+    if (tid < HN && h_lo + tid < Hr) {
+      const int h = h_lo + tid;
       const float m = ss.m_ref[tid], l = ss.l_acc[tid];
       if (partial) {
-        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + tid) * 2;
-        ml[0] = (l > 0.0f) ? m : -INFINITY;
-        ml[1] = l;
+        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + h) * 2;
+        ml[0] = (o_init && l > 0.0f) ? m : -INFINITY;
+        ml[1] = o_init ? l : 0.0f;
       } else if (a.lse) {
-        a.lse[(int64_t)q * Hr + tid] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        a.lse[(int64_t)q * Hr + h] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
     }
-  }
-  __syncthreads();
-  if (done_ok) {
-    float4* dst4 = reinterpret_cast<float4*>(partial ? a.part_o + (((int64_t)q * a.nsplit + split) * Hr) * D
-                                                     : a.out + (int64_t)q * Hr * D);
-    const float4* src4 = reinterpret_cast<const float4*>(so);
-    const int n4 = Hr * D / 4;
-#pragma unroll 4
-    for (int i = tid; i < n4; i += kThreads) dst4[i] = src4[i];
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, G::kTmemCols);
   }
 }
 
-// Merge of the split partials of one query over a 32-dim block: per head the weights
-// 2^(m_s - M) / L, M = max_s m_s, L = sum_s 2^(m_s - M) l_s; partials are [D][H] rows, so the
-// block is read with consecutive threads on consecutive heads and transposed through
-// shared memory for the [H][D] output.
-constexpr int kMergeD = 8;               // output dims per merge CTA
+// Merge of the split partials of one query: per head the weights 2^(m_s - M) / L with
+// M = max_s m_s and L = sum_s 2^(m_s - M) l_s.  Partials are [head][D] rows, so a thread
+// combines one 4-dim group of one head with 16-byte loads, every load in flight at once.
 constexpr int kMaxSplit = 16;
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a, int H, int D) {
-  __shared__ float wgt[kMaxSplit][kN];
-  __shared__ float tile[kN][kMergeD + 1];
-  const int q = blockIdx.x, d0 = blockIdx.y * kMergeD, tid = threadIdx.x;
-  const int ns = a.nsplit;
-  // partial values first: every load of this thread in flight at once
-  const float* base = a.part_o + (int64_t)q * ns * D * H + (int64_t)d0 * H;
-  const int n_el = kMergeD * H;          // <= 512: two per thread
-  float v[2][kMaxSplit];
+  pdl_trigger();
+  pdl_wait();
+  const int q = blockIdx.y, ns = a.nsplit;
+  const int n4 = H * D / 4;                  // 4-dim groups of one partial
+  const int g = blockIdx.x * 256 + threadIdx.x;
+  if (g >= n4) return;
+  const int h = (g * 4) / D;
+  const float4* po = reinterpret_cast<const float4*>(a.part_o + (int64_t)q * ns * H * D) + g;
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml + (int64_t)q * ns * H * 2) + h;
+  float4 v[kMaxSplit];
+  float2 m[kMaxSplit];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int e = tid + 256 * k;
-#pragma unroll
-    for (int s = 0; s < kMaxSplit; ++s)
-      v[k][s] = (e < n_el && s < ns) ? __ldg(base + (int64_t)s * D * H + e) : 0.0f;
-  }
-  if (tid < H) {
-    const float* ml = a.part_ml + (int64_t)q * ns * H * 2;
-    float m[kMaxSplit], l[kMaxSplit];
-#pragma unroll
-    for (int s = 0; s < kMaxSplit; ++s) {
-      m[s] = s < ns ? ml[(s * H + tid) * 2] : -INFINITY;
-      l[s] = s < ns ? ml[(s * H + tid) * 2 + 1] : 0.0f;
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < kMaxSplit; ++s) M = fmaxf(M, m[s]);
-    float L = 0.0f;
-#pragma unroll
-    for (int s = 0; s < kMaxSplit; ++s) {
-      const float w = (m[s] == -INFINITY) ? 0.0f : exp2f(m[s] - M);
-      wgt[s][tid] = w;
-      L += w * l[s];
-    }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-#pragma unroll
-    for (int s = 0; s < kMaxSplit; ++s) wgt[s][tid] *= inv;
-    if (a.lse && blockIdx.y == 0)
-      a.lse[(int64_t)q * H + tid] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int e = tid + 256 * k;
-    if (e < n_el) {
-      const int dd = e / H, h = e - dd * H;
-      float acc = 0.0f;
-#pragma unroll
-      for (int s = 0; s < kMaxSplit; ++s) acc = fmaf(wgt[s][h], v[k][s], acc);
-      tile[h][dd] = acc;
+  for (int s = 0; s < kMaxSplit; ++s) {
+    if (s < ns) {
+      v[s] = __ldg(po + (int64_t)s * n4);
+      m[s] = __ldg(ml + s * H);
+    } else {
+      v[s] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      m[s] = make_float2(-INFINITY, 0.0f);
     }
   }
-  __syncthreads();
-  float* out = a.out + (int64_t)q * H * D + d0;
-  for (int e = tid; e < n_el; e += 256) {
-    const int h = e / kMergeD, dd = e - h * kMergeD;
-    out[(int64_t)h * D + dd] = tile[h][dd];
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) M = fmaxf(M, m[s].x);
+  float L = 0.0f;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) {
+    const float w = (m[s].x == -INFINITY) ? 0.0f : exp2f(m[s].x - M);
+    L = fmaf(w, m[s].y, L);
+    acc.x = fmaf(w, v[s].x, acc.x);
+    acc.y = fmaf(w, v[s].y, acc.y);
+    acc.z = fmaf(w, v[s].z, acc.z);
+    acc.w = fmaf(w, v[s].w, acc.w);
   }
+  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+  reinterpret_cast<float4*>(a.out + (int64_t)q * H * D)[g] =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (a.lse && g * 4 == h * D)
+    a.lse[(int64_t)q * H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------------
@@ -663,13 +635,30 @@ int nsplit_of(int num_q, int n_tiles) {
   return std::max(1, std::min(std::min(n_tiles, kMaxSplit), 512 / std::max(1, num_q)));
 }
 
-size_t attn_smem_bytes(int D) {
-  const size_t q = ((size_t)(D / 64) * kN * 128 + 1023) / 1024 * 1024;
-  return 1024 + q + (size_t)(D / 64) * kTile * 128 + kTile * 128;
+bool attn_shape_ok(int H, int D) {
+  return H >= 1 && H <= 64 && (D == 128 || D == 256 || D == 512);
 }
 
-bool attn_shape_ok(int H, int D) {
-  return H >= 1 && H <= kN && (D == 128 || D == 256 || D == 512);
+// bytes of one staged tile (and of one stash tile): padded code rows, then scale rows
+size_t stage_bytes_of(int D) { return (size_t)kTile * ((size_t)D / 2 + 16 + kScaleStride); }
+
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Heads per CTA: groups of 16 while every CTA of the call fits on the GPU at once (the
+// latency-bound small batches), else 32 (fewer repeated gathers per query).
+int head_group_of(int num_q, int nsplit, int H) {
+  return (int64_t)num_q * nsplit * ((H + 15) / 16) <= sm_count() ? 16 : 32;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
@@ -685,15 +674,34 @@ PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
   return fn;
 }
 
-template <int D>
-cudaError_t launch(const AttnArgs& a, const CUtensorMap& tm, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes(D);
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+// Q as a [num_q][H][D] bf16 map with boxes of 64 dims x HN heads: heads >= H of the last
+// group fall outside the map and read as zero.
+bool make_q_map(CUtensorMap* tm, const uint16_t* q, int num_q, int H, int D, int HN) {
+  auto fn = attn_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)num_q};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)HN, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(q), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int HN>
+cudaError_t launch(AttnArgs a, const uint16_t* q, cudaStream_t st) {
+  using G = Geo<D, HN>;
+  CUtensorMap tm;
+  if (!make_q_map(&tm, q, a.num_q, a.H, D, HN)) return cudaErrorInvalidValue;
+  a.hsplit = (a.H + HN - 1) / HN;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, HN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<D><<<dim3(a.nsplit, a.num_q), kThreads, smem, st>>>(tm, a);
-  if (a.nsplit > 1) attn_merge_kernel<<<dim3(a.num_q, D / kMergeD), 256, 0, st>>>(a, a.H, D);
-  return cudaGetLastError();
+  e = launch_pdl(attn_tc_kernel<D, HN>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
+                 (size_t)G::kSmem, st, tm, a);
+  if (e != cudaSuccess || a.nsplit <= 1) return e;
+  return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + 255) / 256, a.num_q), dim3(256), 0, st,
+                    a, a.H, D);
 }
 
 }  // namespace
@@ -703,7 +711,7 @@ using namespace csa2;
 
 extern "C" size_t csa2_sparse_attn_stash_bytes(int32_t num_q, int32_t D, int32_t topk) {
   if (num_q < 0 || D < 1 || topk < 0) return 0;
-  return (size_t)num_q * ((topk + kTile - 1) / kTile) * (size_t)D * 256;
+  return (size_t)num_q * ((topk + kTile - 1) / kTile) * stage_bytes_of(D);
 }
 
 extern "C" size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
@@ -741,12 +749,12 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
     return kv_stash && (reinterpret_cast<uintptr_t>(kv_stash) & 15) ? CSA2_ERR_INVALID_ARG
                                                                     : CSA2_ERR_CAPACITY;
   if (num_q == 0) return CSA2_OK;
-  if ((int64_t)num_q * H > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;
+  if (num_q > 65535) return CSA2_ERR_UNSUPPORTED;       // queries are a grid dimension
   if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
   if (topk > 0 && (!indices || !kv_codes || !kv_scales || cap_rows <= 0)) return CSA2_ERR_INVALID_ARG;
   if (window > 0 && (!swa_kv || !swa_start || swa_rows < 0)) return CSA2_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 15) ||
-      (reinterpret_cast<uintptr_t>(kv_scales) & 1) || (reinterpret_cast<uintptr_t>(swa_kv) & 15) ||
+      (reinterpret_cast<uintptr_t>(kv_scales) & 15) || (reinterpret_cast<uintptr_t>(swa_kv) & 15) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(out) & 15))
     return CSA2_ERR_INVALID_ARG;
   AttnArgs a{};
@@ -772,21 +780,11 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   a.part_ml = reinterpret_cast<float*>(ws + off);
   a.out = out; a.lse = lse;
 
-  auto fn = attn_encode_fn();
-  if (!fn) return CSA2_ERR_CUDA;
-  CUtensorMap tm;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_q * H};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)H};
-  cuuint32_t estr[2] = {1u, 1u};
-  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), dims, strides, box,
-         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return CSA2_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
+  const bool g16 = head_group_of(num_q, a.nsplit, H) == 16;
   cudaError_t e = cudaSuccess;
-  if (D == 128) e = launch<128>(a, tm, st);
-  else if (D == 256) e = launch<256>(a, tm, st);
-  else e = launch<512>(a, tm, st);
+  if (D == 128) e = g16 ? launch<128, 16>(a, q, st) : launch<128, 32>(a, q, st);
+  else if (D == 256) e = g16 ? launch<256, 16>(a, q, st) : launch<256, 32>(a, q, st);
+  else e = g16 ? launch<512, 16>(a, q, st) : launch<512, 32>(a, q, st);
   return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

@@ -136,6 +136,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   uint32_t* shist = rowp + ((a.num_q + 1 + 31) & ~31);                             // [kHistBins]
   uint32_t* sbhist = shist + kHistBins;                                            // [kHistBins]
 
+  // set-up that reads no global memory (it overlaps the previous kernel's tail)
+  pdl_trigger();
+  for (int i = tid; i < 2 * kHistBins; i += kScoreThreads) shist[i] = 0;
+  if (tid == 0) {
+    rowp[0] = 0;
+    for (int s = 0; s < S; ++s) { mbar_init(&ss.full[s], 1); mbar_init(&ss.empty[s], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&ss.tfull[i], 1); mbar_init(&ss.tempty[i], 4); }
+    ss.abort = 0;
+    fence_barrier_init();
+  }
+  // padding rows of the B operand (heads >= H_I) must read as zero; TMA never writes them
+  if (a.H_I < a.n_pad) {
+    const uint32_t pad = (uint32_t)(a.n_pad - a.H_I) * 128;
+    for (int s = 0; s < S; ++s) {
+      uint8_t* b = base + (size_t)s * stage_bytes + a_bytes;
+      for (uint32_t i = tid * 16; i < (uint32_t)halves * pad; i += kScoreThreads * 16) {
+        const uint32_t h = i / pad, o = i % pad;
+        *reinterpret_cast<uint4*>(b + h * b_half + (uint32_t)a.H_I * 128 + o) = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  if (warp == 1) { tmem_alloc(&ss.tmem_base, a.n_pad * 2 < 32 ? 32 : a.n_pad * 2); tmem_relinquish(); }
+  pdl_wait();
+
   // active tiles of every query, then their exclusive prefix
   if (kGather) {
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = 0;
@@ -172,25 +196,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   } else {
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles_of<kGather>(a, a.q0 + i);
   }
-  for (int i = tid; i < 2 * kHistBins; i += kScoreThreads) shist[i] = 0;
-  if (tid == 0) {
-    rowp[0] = 0;
-    for (int s = 0; s < S; ++s) { mbar_init(&ss.full[s], 1); mbar_init(&ss.empty[s], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&ss.tfull[i], 1); mbar_init(&ss.tempty[i], 4); }
-    ss.abort = 0;
-    fence_barrier_init();
-  }
-  // padding rows of the B operand (heads >= H_I) must read as zero; TMA never writes them
-  if (a.H_I < a.n_pad) {
-    const uint32_t pad = (uint32_t)(a.n_pad - a.H_I) * 128;
-    for (int s = 0; s < S; ++s) {
-      uint8_t* b = base + (size_t)s * stage_bytes + a_bytes;
-      for (uint32_t i = tid * 16; i < (uint32_t)halves * pad; i += kScoreThreads * 16) {
-        const uint32_t h = i / pad, o = i % pad;
-        *reinterpret_cast<uint4*>(b + h * b_half + (uint32_t)a.H_I * 128 + o) = make_uint4(0, 0, 0, 0);
-      }
-    }
-  }
   __syncthreads();
   if (warp == 0) {
     uint32_t carry = 0;
@@ -205,7 +210,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
   }
-  if (warp == 1) { tmem_alloc(&ss.tmem_base, a.n_pad * 2 < 32 ? 32 : a.n_pad * 2); tmem_relinquish(); }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -634,6 +638,15 @@ __device__ void final_select(const SelProblem& p, int r, const Top& tp, const Sr
   }
 }
 
+// Clears the per-call counters and histograms of the workspace (a kernel rather than a
+// memset, so that the launches of one call chain without gaps).
+__global__ void __launch_bounds__(256) ws_zero_kernel(uint4* p, uint32_t n16) {
+  pdl_trigger();
+  pdl_wait();
+  for (uint32_t i = blockIdx.x * 256u + threadIdx.x; i < n16; i += gridDim.x * 256u)
+    p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 constexpr int kStageCap = 12288;       // candidates staged in shared memory (96 KB)
 
 __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a) {
@@ -646,6 +659,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   __shared__ __align__(16) uint32_t hsm[2048];
   __shared__ uint32_t pre[kMaxListChunks + 1];
   __shared__ uint32_t soff[kMaxListChunks];  // list offset of each chunk's candidates
+  pdl_trigger();
+  pdl_wait();
   const SelProblem& p = a.p[blockIdx.z];
   const int r = blockIdx.y, c = blockIdx.x;
   if (r >= p.num_rows) return;
@@ -893,8 +908,13 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   int* status = reinterpret_cast<int*>(wsb);
   Seqs sq{seqs.seq_start, seqs.seq_len, q_visible, seqs.q_per_seq, max_visible, status};
 
-  if (cudaMemsetAsync(wsb + L.zero_lo, 0, L.zero_hi - L.zero_lo, stream) != cudaSuccess)
-    return CSA2_ERR_CUDA;
+  {
+    const uint32_t n16 = (uint32_t)((L.zero_hi - L.zero_lo) / 16);   // both ends 256-aligned
+    const unsigned blocks = std::max(1u, std::min(64u, (n16 + 255u) / 256u));
+    if (launch_pdl(ws_zero_kernel, dim3(blocks), dim3(256), 0, stream,
+                   reinterpret_cast<uint4*>(wsb + L.zero_lo), n16) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+  }
 
   // ---- scores (+ first-digit histograms) ----
   CUtensorMap tm_k, tm_q;
@@ -932,8 +952,9 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return CSA2_ERR_CUDA;
-    kern<<<grid, kScoreThreads, smem, stream>>>(tm_k, tm_q, sa);
-    if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+    if (launch_pdl(kern, dim3(grid), dim3(kScoreThreads), smem, stream, tm_k, tm_q, sa) !=
+        cudaSuccess)
+      return CSA2_ERR_CUDA;
   }
 
   // ---- selection ----
@@ -976,8 +997,9 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sel_smem) != cudaSuccess)
     return CSA2_ERR_CUDA;
-  select_kernel<<<grid, kSelThreads, sel_smem, stream>>>(sel);
-  return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+  return launch_pdl(select_kernel, grid, dim3(kSelThreads), sel_smem, stream, sel) == cudaSuccess
+             ? CSA2_OK
+             : CSA2_ERR_CUDA;
 }
 
 csa2_status_t check_common(const uint16_t* qI, const float* w, int num_q, int H_I, int d_I,

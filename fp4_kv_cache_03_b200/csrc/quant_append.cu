@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(256) quant_append_kernel(
     const float* __restrict__ x, int rows, int D, const int64_t* __restrict__ dst_row,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int64_t cap,
     const uint16_t* __restrict__ kin, uint16_t* __restrict__ kout, int d_I, int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int gpr = D >> 4;                      // channel groups per row
   const int cpr = kin ? (d_I >> 3) : 0;        // 16-byte chunks of indexer K per row
   const int64_t n_q = (int64_t)rows * gpr;
@@ -105,8 +107,9 @@ extern "C" csa2_status_t csa2_quant_append(const float* x, int32_t rows, int32_t
   const int threads = 256;
   const int64_t blocks = (n + threads - 1) / threads;
   if (blocks > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;
-  csa2::quant_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+  const cudaError_t e = csa2::launch_pdl(
+      csa2::quant_append_kernel, dim3((unsigned)blocks), dim3(threads), 0, (cudaStream_t)stream,
       x, rows, D, dst_row, kv_codes, kv_scales, cap_rows, idx_k_in, idx_k, idx_k_in ? d_I : 0,
       static_cast<int*>(workspace));
-  return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+  return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

@@ -17,7 +17,10 @@
  *     no state between calls.
  *   - bf16 data is passed as its raw 16-bit patterns (uint16_t).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
- *     enqueues work on it and returns; results are ready when the stream is.
+ *     enqueues work on it and returns; results are ready when the stream is.  Kernels
+ *     are launched as programmatic dependents of the work before them in the stream: a
+ *     kernel may start its set-up while the previous kernel still runs, but reads no
+ *     memory until that kernel has completed, so stream order is kept.
  *   - Shape, pointer and workspace-size errors are detected on the host and returned
  *     before anything is enqueued.  Values that live in device memory (lengths, row
  *     ids, indices) are checked by the kernels: a bad value is skipped and the first
@@ -199,15 +202,17 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   lse = -inf.  The two sets share one softmax; a row in both counts twice.
  * Cross-layer reuse ([SURV] §2.2.2, [MTP] "CSA2：…": a Reuse layer takes the main KV and the
  * latest Top-K of an earlier layer): with a non-NULL `kv_stash`,
- *   - mode FULL or REINDEX also stores the dequantised selected rows (bf16, in the kernel's
- *     tile layout) into kv_stash;
+ *   - mode FULL or REINDEX also stores the selected rows' FP4 codes and scales (per
+ *     128-slot tile, in the kernel's staging layout) into kv_stash;
  *   - mode REUSE takes the selected rows from kv_stash instead of the FP4 cache.  The
  *     stash must hold the rows of exactly these indices for these queries, as written by
  *     the latest FULL/REINDEX call with the same num_q, D and topk; the window rows are
  *     always read from swa_kv.  Results equal those of a stateless call.
  *   With kv_stash == NULL every mode reads the FP4 cache (the call is stateless).
- *   q         device bf16 [num_q][H][D]        1 <= H <= 64, D in {128, 256, 512} (other
- *             shapes return CSA2_ERR_UNSUPPORTED); base 16-byte aligned
+ *   q         device bf16 [num_q][H][D]        1 <= H <= 64, D in {128, 256, 512},
+ *             num_q <= 65535 (other shapes return CSA2_ERR_UNSUPPORTED); base 16-byte
+ *             aligned
+ *   kv_codes, kv_scales  the cache (layout above), both 16-byte aligned
  *   indices   device int32 [num_q][topk]       0 <= topk <= 2048
  *   swa_kv    device bf16 [swa_rows][D];  swa_start device int64 [num_seqs] (may be
  *             negative: only rows of window positions are read)

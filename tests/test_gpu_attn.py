@@ -99,7 +99,7 @@ def test_decoder_group_128k_attention():
 
 
 def test_reuse_stash_equals_stateless():
-    """Reuse layers reading the stashed bf16 rows give bit-identical results to Reuse
+    """Reuse layers reading the stashed FP4 rows give bit-identical results to Reuse
     layers that gather and dequantise the FP4 rows again; Reindex layers refresh it."""
     from fp4_kv_cache_03_b200.workload import DeviceWorkload
     W = small_workload(lengths=(3000, 9000), D=512, H=64, H_I=16, d_I=128, topk=256,
