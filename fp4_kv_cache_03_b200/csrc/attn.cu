@@ -10,10 +10,12 @@
 // Per tile:
 //   stage    the selected rows' FP4 codes and scales are copied with cp.async (row-
 //            contiguous, 16-byte pieces) into a staging area -- or, in a Reuse layer with
-//            a stash, come back as one bulk copy of the stage image that the group's
-//            Full / Reindex call stored; window rows go by cp.async straight into the tile;
+//            a stash, come back as one bulk copy of the stage image (with the slots'
+//            validity) that the group's Full / Reindex call stored, so that the layer
+//            reads no indices; window rows go by cp.async straight into the tile;
 //   dequant  all 8 warps decode the staged rows to bf16 (exact: a 2-bit-mantissa code times
-//            a 4-bit-mantissa scale) into a 128-byte-swizzled [128 keys x D] tile;
+//            a 4-bit-mantissa scale) into the KV tile: D/16 slices of [128 keys x 32 B]
+//            with the 32-byte swizzle, which both MMAs read as contiguous 4 KB blocks;
 //   S^T      one thread issues tcgen05.mma: S^T[key, head] = KV[key, :] . Q[head, :]
 //            (M = 128 keys, N = the CTA's heads, K = D; Q arrives once by TMA);
 //   softmax  all 8 warps read S^T from TMEM (one key per thread, half the heads per warp),
@@ -29,6 +31,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -77,17 +80,23 @@ struct Geo {
   static constexpr int kChunks = D / 64;               // 64-element (128-byte) column chunks
   static constexpr int kSlabs = D / 128;               // O^T slabs of 128 dims (MMA M)
   static constexpr uint32_t kQChunk = HN * 128;        // Q chunk: [HN rows][128 B]
-  static constexpr uint32_t kKVChunk = kTile * 128;    // KV chunk: [128 keys][128 B]
+  // KV tile: D/16 slices of 16 dims, each [128 keys][32 B] with the 32-byte swizzle, so
+  // that one MMA K-step (S^T) or one 16-dim chunk of V^T (O^T) is a contiguous 4 KB
+  static constexpr uint32_t kKVSlice = kTile * 32;
+  static constexpr uint32_t kKVBytes = (D / 16) * kKVSlice;
   static constexpr uint32_t kPChunk = HN * 128;        // P chunk: [HN heads][64 keys]
   static constexpr uint32_t kCodeStride = D / 2 + 16;  // staged code row (padded: no bank conflicts)
   static constexpr uint32_t kStageCodes = kTile * kCodeStride;
-  static constexpr uint32_t kStageBytes = kStageCodes + kTile * kScaleStride;
+  static constexpr uint32_t kStageValid = kStageCodes + kTile * kScaleStride;  // 1 byte per slot
+  static constexpr uint32_t kStageBytes = kStageValid + kTile;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = (kChunks * kQChunk + 1023) / 1024 * 1024;
-  static constexpr uint32_t kOffP = kOffKV + kChunks * kKVChunk;
+  static constexpr uint32_t kOffP = kOffKV + kKVBytes;
   static constexpr uint32_t kOffStage = kOffP + (2 * kPChunk + 1023) / 1024 * 1024;
   static constexpr uint32_t kSmem = 1024 + kOffStage + kStageBytes;
-  static constexpr uint32_t kTmemCols = (HN + kSlabs * HN) <= 128 ? 128 : 256;
+  // S^T as kSAcc partial accumulators (independent MMA chains), then the O^T slabs
+  static constexpr int kSAcc = 4;
+  static constexpr uint32_t kTmemCols = (kSAcc * HN + kSlabs * HN) <= 128 ? 128 : 256;
   static_assert(kStageBytes % 16 == 0 && D / 16 <= kScaleStride, "stage layout");
 };
 
@@ -184,14 +193,19 @@ __device__ __forceinline__ void warp_reduce_heads(float* v, int lane) {
 
 template <int D, int HN>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_swa, const AttnArgs a) {
   using G = Geo<D, HN>;
   constexpr int kChunks = G::kChunks, kSlabs = G::kSlabs;
   constexpr int HW = HN / 2;                 // heads per warp in softmax and epilogue
   constexpr int kParts = D / 32;             // 16-byte code pieces (32 values) of a row
   constexpr int kRowsPerIter = kThreads / kParts;
   constexpr int kIters = kTile / kRowsPerIter;
-  constexpr uint32_t kKVChunk = G::kKVChunk;
+  constexpr uint32_t kKVSlice = G::kKVSlice;
+  // byte offset of 16-byte unit u (dims 8u .. 8u+7) of key row r in the KV tile
+  auto kv_off = [](int r, int u) -> uint32_t {
+    return (uint32_t)(u >> 1) * kKVSlice + (uint32_t)r * 32 + ((uint32_t)((u & 1) ^ ((r >> 2) & 1)) << 4);
+  };
   const int Hr = a.H;
 
   extern __shared__ uint8_t smem_raw[];
@@ -204,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = base + G::kOffP;
   uint8_t* sStage = base + G::kOffStage;
   uint8_t* sScale = sStage + G::kStageCodes;
+  uint8_t* sValid = sStage + G::kStageValid;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3;                 // TMEM lane quadrant of this warp
@@ -225,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ss.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
+    if (a.window > 0 && a.swa_rows > 0) tma_prefetch_desc(&tm_swa);
   }
   if (tid < HN) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
   if (warp == 0) { tmem_alloc(&ss.tmem_base, G::kTmemCols); tmem_relinquish(); }
@@ -239,7 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t my_idx = 0;
   auto fetch_idx = [&](int t) {
     const int slot = t * kTile + tid;
-    if (tid < kTile && slot < a.topk) my_idx = __ldg(a.indices + (int64_t)q * a.topk + slot);
+    const bool stashed = a.stash != nullptr && a.mode == CSA2_MODE_REUSE && t < a.n_idx_tiles;
+    if (tid < kTile && slot < a.topk && !stashed) my_idx = __ldg(a.indices + (int64_t)q * a.topk + slot);
   };
   if (t_begin < t_end) fetch_idx(t_begin);
 
@@ -254,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem_base;
-  const uint32_t tS = tmem;                  // S^T: columns [0, HN)
-  const uint32_t tO = tmem + HN;             // O^T slab j: columns [HN + j HN, HN + (j+1) HN)
+  const uint32_t tS = tmem;                  // S^T partial a: columns [a HN, (a+1) HN)
+  const uint32_t tO = tmem + G::kSAcc * HN;  // O^T slab j: HN columns from tO + j HN
   const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
   const uint32_t idesc_s = idesc_bf16(kTile, HN);                  // KV, Q both K-major
@@ -270,6 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool from_stash = stash_tile && a.mode == CSA2_MODE_REUSE;
     const bool to_stash = stash_tile && a.mode != CSA2_MODE_REUSE && hg == 0;
     uint8_t* stile = stash_tile ? a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStageBytes : nullptr;
+    // a tile of window slots only comes in by TMA: D/16 boxes of [128 rows x 16 dims], each
+    // one slice of the tile (rows outside the window are masked, and zeroed below)
+    const bool win_tile = t * kTile >= a.topk;
     // the previous tile's O^T MMA and stash store must be done before its buffers are rewritten
     if (store_pending && tid == 0) bulk_wait_read();
     if (o_pending) {
@@ -282,16 +302,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
     }
     store_pending = false;
-    if (from_stash && tid == 0) {            // needs no index: goes out first
+    if (tid == 0 && from_stash) {            // needs no index: goes out first
       mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
       bulk_g2s(sStage, stile, G::kStageBytes, &ss.bar_kv);
+    } else if (tid == 0 && win_tile) {
+      if (a.swa_rows > 0) {
+        // (rows are below 2^31; a start that far outside the map loads zeros only)
+        const int64_t y = wrow0 + ((int64_t)t * kTile - a.topk);
+        const int32_t y0 = (y < -(int64_t)(1 << 30) || y > (int64_t)0x7FFFFF00) ? -(1 << 30) : (int32_t)y;
+        mbar_arrive_expect_tx(&ss.bar_kv, (uint32_t)(D / 16) * kKVSlice);
+        for (int sl = 0; sl < D / 16; ++sl)
+          tma_load_2d(sKV + sl * kKVSlice, &tm_swa, sl * 16, y0, &ss.bar_kv);
+      } else {
+        mbar_arrive(&ss.bar_kv);             // no rows: every slot is masked and zeroed
+      }
     }
     // ------------------------- slots -> sources (one thread per row) -------------------------
+    bool ok = true;
+    if (from_stash && tid < kTile) ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
+    if (from_stash) ph_kv ^= 1;
     if (tid < kTile) {
       const int slot = t * kTile + tid;
       int kind = 0;
       int64_t src = 0;
-      if (slot < a.topk) {
+      if (slot < a.topk && from_stash) {
+        kind = sValid[tid] ? 1 : 0;              // rows are in the stage already
+      } else if (slot < a.topk) {
         const int p = my_idx;
         if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
           kind = 1;
@@ -312,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ss.kind[tid] = kind;
       ss.src[tid] = src;
+      if (to_stash && slot < a.topk) sValid[tid] = kind != 0;
     }
-    __syncthreads();
+    if (__syncthreads_or(!ok)) break;
     if (t + 1 < t_end) fetch_idx(t + 1);
     // ------------------------- loads (a row's threads are contiguous) -------------------------
     {
@@ -330,12 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             if (lp == 0) cp_async8(sScale + r * kScaleStride, a.scales + grow * (D / 16));
           }
-        } else if (kind == 2) {
+        } else if (kind == 2 && !win_tile) {
           const uint16_t* src = a.swa + ss.src[r] * D;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int u = 4 * lp + i;
-            cp_async16(sKV + (u >> 3) * kKVChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4), src + u * 8);
+            cp_async16(sKV + kv_off(r, u), src + u * 8);
           }
         } else if (kind == 0 && to_stash && t * kTile + r < a.topk) {
           // an index slot without a row is stored as zero codes and scales
@@ -350,8 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     cp_async_wait_all();
-    bool ok = true;
-    if (from_stash) {
+    if (win_tile) {
       ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
       ph_kv ^= 1;
     }
@@ -366,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ------------------------- dequantise into the swizzled tile -------------------------
     // consecutive threads take consecutive rows: the 8 threads of a quarter warp then store
-    // to 8 different rows, whose 128-byte swizzle puts their 16-byte units in 8 bank groups
+    // one 16-byte unit of each of 8 consecutive rows of a slice, which the 32-byte swizzle
+    // spreads over all 32 banks
     {
       const int rsub = tid % kRowsPerIter;
       const int part = tid / kRowsPerIter;
@@ -374,7 +411,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < kIters; ++it) {
         const int r = it * kRowsPerIter + rsub;
         const int kind = ss.kind[r];
-        uint8_t* row_smem = sKV + r * 128;
         // a stash holds zero codes for index slots without a row
         const bool dec = from_stash ? (t * kTile + r < a.topk) : (kind == 1);
         if (dec) {
@@ -392,14 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ow[k], s2);
             const int u = 4 * part + i;
-            *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) = o;
+            *reinterpret_cast<uint4*>(sKV + kv_off(r, u)) = o;
           }
         } else if (kind == 0) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int u = 4 * part + i;
-            *reinterpret_cast<uint4*>(row_smem + (u >> 3) * kKVChunk + (((u & 7) ^ (r & 7)) << 4)) =
-                make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sKV + kv_off(r, u)) = make_uint4(0, 0, 0, 0);
           }
         }
       }
@@ -414,13 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!q_ready) { okq = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = okq; }
       if (okq) {
         tc_fence_after();
-        const uint64_t kv_desc_k = sdesc_sw128(smem_u32(sKV), 16, 1024);   // KV as K-major A
+        const uint64_t kv_desc_k = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);  // KV as K-major A
         const uint64_t q_desc_k = sdesc_sw128(smem_u32(sQ), 16, 1024);     // Q as K-major B
+        // K-step k accumulates into partial k mod kSAcc: kSAcc independent chains
 #pragma unroll 4
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (uint32_t)(k >> 2) * kKVChunk + (k & 3) * 32;
+          const uint32_t off = (uint32_t)k * kKVSlice;
           const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunk + (k & 3) * 32;
-          umma_bf16(tS, kv_desc_k + (off >> 4), q_desc_k + (qoff >> 4), idesc_s, k > 0 ? 1u : 0u);
+          umma_bf16(tS + (uint32_t)(k % G::kSAcc) * HN, kv_desc_k + (off >> 4),
+                    q_desc_k + (qoff >> 4), idesc_s, k >= G::kSAcc ? 1u : 0u);
         }
         umma_commit(&ss.bar_s);
       }
@@ -435,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_s ^= 1;
     if (!ok) break;
     tc_fence_after();
-    tmem_ldn<HW>(tS + lane_base + h0, v);
+    tmem_ld_sum4<HW>(tS + lane_base + h0, HN, v);   // S^T = the sum of the partials
     {
       const bool valid = ss.kind[r] != 0;
 #pragma unroll
@@ -503,14 +540,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ O^T += V^T . P^T ------------------------------
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t kv_desc_mn = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);  // V^T, MN-major A
+      const uint64_t kv_desc_mn = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);    // V^T, MN-major A
       const uint64_t p_desc_k = sdesc_sw128(smem_u32(sP), 16, 1024);           // P, K-major B
-#pragma unroll 1
-      for (int j = 0; j < kSlabs; ++j) {
-#pragma unroll 4
-        for (int k = 0; k < kTile / 16; ++k) {
-          const uint32_t off = (uint32_t)(2 * j) * kKVChunk + k * 2048;
-          const uint32_t poff = (uint32_t)(k >> 2) * G::kPChunk + (k & 3) * 32;
+      // key steps outermost: consecutive MMAs go to the kSlabs independent slabs
+#pragma unroll 2
+      for (int k = 0; k < kTile / 16; ++k) {
+        const uint32_t poff = (uint32_t)(k >> 2) * G::kPChunk + (k & 3) * 32;
+#pragma unroll
+        for (int j = 0; j < kSlabs; ++j) {
+          const uint32_t off = (uint32_t)(8 * j) * kKVSlice + k * 512;   // 16 keys = 2 atoms
           umma_bf16(tO + j * HN, kv_desc_mn + (off >> 4), p_desc_k + (poff >> 4), idesc_o,
                     (o_init || k > 0) ? 1u : 0u);
         }
@@ -639,8 +677,9 @@ bool attn_shape_ok(int H, int D) {
   return H >= 1 && H <= 64 && (D == 128 || D == 256 || D == 512);
 }
 
-// bytes of one staged tile (and of one stash tile): padded code rows, then scale rows
-size_t stage_bytes_of(int D) { return (size_t)kTile * ((size_t)D / 2 + 16 + kScaleStride); }
+// bytes of one staged tile (and of one stash tile): padded code rows, scale rows, then one
+// validity byte per slot
+size_t stage_bytes_of(int D) { return (size_t)kTile * ((size_t)D / 2 + 16 + kScaleStride + 1); }
 
 int sm_count() {
   static std::atomic<int> cached[64];
@@ -688,17 +727,35 @@ bool make_q_map(CUtensorMap* tm, const uint16_t* q, int num_q, int H, int D, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The window rows as a [swa_rows][D] bf16 map with boxes of 16 dims x 128 rows and the
+// 32-byte swizzle: one box is one slice of the KV tile.  Rows outside the map read as zero.
+bool make_swa_map(CUtensorMap* tm, const uint16_t* swa, int64_t rows, int D) {
+  auto fn = attn_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {16u, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(swa), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int HN>
 cudaError_t launch(AttnArgs a, const uint16_t* q, cudaStream_t st) {
   using G = Geo<D, HN>;
   CUtensorMap tm;
   if (!make_q_map(&tm, q, a.num_q, a.H, D, HN)) return cudaErrorInvalidValue;
+  CUtensorMap tm_swa;
+  std::memset(&tm_swa, 0, sizeof(tm_swa));  // not read without window slots
+  if (a.window > 0 && a.swa_rows > 0 && !make_swa_map(&tm_swa, a.swa, a.swa_rows, D))
+    return cudaErrorInvalidValue;
   a.hsplit = (a.H + HN - 1) / HN;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, HN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(attn_tc_kernel<D, HN>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
-                 (size_t)G::kSmem, st, tm, a);
+                 (size_t)G::kSmem, st, tm, tm_swa, a);
   if (e != cudaSuccess || a.nsplit <= 1) return e;
   return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + 255) / 256, a.num_q), dim3(256), 0, st,
                     a, a.H, D);
@@ -753,6 +810,7 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
   if (topk > 0 && (!indices || !kv_codes || !kv_scales || cap_rows <= 0)) return CSA2_ERR_INVALID_ARG;
   if (window > 0 && (!swa_kv || !swa_start || swa_rows < 0)) return CSA2_ERR_INVALID_ARG;
+  if (swa_rows > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;    // window rows are TMA coordinates
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 15) ||
       (reinterpret_cast<uintptr_t>(kv_scales) & 15) || (reinterpret_cast<uintptr_t>(swa_kv) & 15) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(out) & 15))

@@ -76,6 +76,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// raise the expected transaction bytes of the current phase without arriving
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -219,6 +225,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   return d;
 }
 
+// The same descriptor for the 32-byte-swizzled layout (atoms of 8 rows x 32 B):
+// K-major: 32-byte rows (16 bf16 of K), 8-row groups SBO apart; MN-major: 16 MN-contiguous
+// elements per 32-B row, 8 K-rows per atom, LBO between 16-element MN chunks, SBO between
+// 8-row K groups.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t smem_addr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)6 << 61;  // SWIZZLE_32B
+  return d;
+}
+
 // 32 TMEM lanes x 32 bits, 16 consecutive columns starting at `taddr`; one value per
 // column for the calling thread's lane.  Whole warp, waits for completion.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -301,6 +322,70 @@ __device__ __forceinline__ void tmem_ldn(uint32_t taddr, float* v) {
   }
 #pragma unroll
   for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Sum of 4 groups of N (8 or 16) consecutive TMEM columns, group a starting at
+// taddr + a * stride: all loads in flight, one wait (as in tmem_ld32).
+template <int N>
+__device__ __forceinline__ void tmem_ld_sum4(uint32_t taddr, uint32_t stride, float* v) {
+  static_assert(N == 8 || N == 16, "8 or 16 columns");
+  uint32_t r[4][N];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    if constexpr (N == 8) {
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(r[g][0]), "=r"(r[g][1]), "=r"(r[g][2]), "=r"(r[g][3]), "=r"(r[g][4]),
+                     "=r"(r[g][5]), "=r"(r[g][6]), "=r"(r[g][7])
+                   : "r"(taddr + g * stride));
+    } else {
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+          "%13,%14,%15}, [%16];"
+          : "=r"(r[g][0]), "=r"(r[g][1]), "=r"(r[g][2]), "=r"(r[g][3]), "=r"(r[g][4]),
+            "=r"(r[g][5]), "=r"(r[g][6]), "=r"(r[g][7]), "=r"(r[g][8]), "=r"(r[g][9]),
+            "=r"(r[g][10]), "=r"(r[g][11]), "=r"(r[g][12]), "=r"(r[g][13]), "=r"(r[g][14]),
+            "=r"(r[g][15])
+          : "r"(taddr + g * stride));
+    }
+  }
+  // one wait; every destination register is named so that no use moves above it
+  if constexpr (N == 8) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]),
+                   "+r"(r[0][5]), "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[1][0]), "+r"(r[1][1]),
+                   "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]), "+r"(r[1][6]),
+                   "+r"(r[1][7]), "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]),
+                   "+r"(r[2][4]), "+r"(r[2][5]), "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[3][0]),
+                   "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]),
+                   "+r"(r[3][6]), "+r"(r[3][7])
+                 :
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]),
+                   "+r"(r[0][5]), "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[0][8]), "+r"(r[0][9]),
+                   "+r"(r[0][10]), "+r"(r[0][11]), "+r"(r[0][12]), "+r"(r[0][13]),
+                   "+r"(r[0][14]), "+r"(r[0][15]), "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]),
+                   "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]), "+r"(r[1][6]), "+r"(r[1][7]),
+                   "+r"(r[1][8]), "+r"(r[1][9]), "+r"(r[1][10]), "+r"(r[1][11]),
+                   "+r"(r[1][12]), "+r"(r[1][13]), "+r"(r[1][14]), "+r"(r[1][15])
+                 :
+                 : "memory");
+    asm volatile("" : "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]),
+                      "+r"(r[2][5]), "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[2][8]), "+r"(r[2][9]),
+                      "+r"(r[2][10]), "+r"(r[2][11]), "+r"(r[2][12]), "+r"(r[2][13]),
+                      "+r"(r[2][14]), "+r"(r[2][15]), "+r"(r[3][0]), "+r"(r[3][1]),
+                      "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]), "+r"(r[3][6]),
+                      "+r"(r[3][7]), "+r"(r[3][8]), "+r"(r[3][9]), "+r"(r[3][10]),
+                      "+r"(r[3][11]), "+r"(r[3][12]), "+r"(r[3][13]), "+r"(r[3][14]),
+                      "+r"(r[3][15])
+                 :
+                 : "memory");
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    v[i] = (__uint_as_float(r[0][i]) + __uint_as_float(r[1][i])) +
+           (__uint_as_float(r[2][i]) + __uint_as_float(r[3][i]));
 }
 
 // store 16 consecutive columns of the calling thread's lane (whole warp); call

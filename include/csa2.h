@@ -214,8 +214,10 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *             aligned
  *   kv_codes, kv_scales  the cache (layout above), both 16-byte aligned
  *   indices   device int32 [num_q][topk]       0 <= topk <= 2048
- *   swa_kv    device bf16 [swa_rows][D];  swa_start device int64 [num_seqs] (may be
- *             negative: only rows of window positions are read)
+ *   swa_kv    device bf16 [swa_rows][D], swa_rows < 2^31;  swa_start device int64
+ *             [num_seqs] (may be negative).  Only rows of window positions take part;
+ *             other rows inside [0, swa_rows) may be read by the tile loads but are
+ *             masked and do not change the result.
  *   q_pos     device int64 [num_q]
  *   window    0 .. 1024
  *   out       device fp32 [num_q][H][D];  lse device fp32 [num_q][H] or NULL

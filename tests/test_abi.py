@@ -98,8 +98,9 @@ def test_host_checks_attention(L):
     assert call(mode=7) == csa2.ERR_INVALID_ARG
     assert call(stash=ctypes.c_void_p(0x200000), stash_bytes=16) == csa2.ERR_CAPACITY
     assert call(stash=ctypes.c_void_p(0x200008), stash_bytes=1 << 30) == csa2.ERR_INVALID_ARG
-    # 4 tiles of 128 staged rows: padded codes (256 + 16 B) and a 48-byte scale row
-    assert L.csa2_sparse_attn_stash_bytes(1, 512, 512) == 4 * 128 * (256 + 16 + 48)
+    # 4 tiles of 128 staged rows: padded codes (256 + 16 B), a 48-byte scale row and a
+    # validity byte
+    assert L.csa2_sparse_attn_stash_bytes(1, 512, 512) == 4 * 128 * (256 + 16 + 48 + 1)
 
 
 def test_device_query_without_gpu_is_harmless(L):
