@@ -37,6 +37,7 @@ constexpr int kSelChunk = 8192;        // keys per select CTA
 constexpr int kHistBins = 2048;        // first digit: key bits 31..21
 constexpr int kMaxRowsPerLaunch = 4096;
 constexpr int kMaxListChunks = 1024;   // rows longer than this many chunks stream their keys
+constexpr int kSelSingle = 16384;      // rows up to this long are selected by one CTA
 
 // ---------------------------------------------------------------------------------
 // visibility
@@ -402,6 +403,7 @@ struct SelProblem {
   uint32_t* fill;       // [rows] candidates appended so far
   uint32_t* done;       // [rows] chunks finished
   int chunks;           // grid bound on chunks per row
+  int single;           // stride <= kSelSingle: one CTA selects the whole row in shared memory
 };
 struct SelArgs {
   SelProblem p[2];
@@ -575,7 +577,7 @@ struct GlobalSource {
 // Exact selection of the row's Top-K from its candidates (any source in position order).
 template <class Src>
 __device__ void final_select(const SelProblem& p, int r, const Top& tp, const Src& src,
-                             uint32_t* red, uint32_t* hsm) {
+                             uint32_t* red, uint32_t* hsm, const int32_t* pool_s = nullptr) {
   const int tid = threadIdx.x;
   const uint32_t k = (uint32_t)p.k;
   int32_t* out = p.out + (int64_t)r * p.out_stride;
@@ -632,7 +634,9 @@ __device__ void final_select(const SelProblem& p, int r, const Top& tp, const Sr
     if (sel) {
       const uint32_t pos = src.pos_at_ordered(g, c);
       int32_t v = (int32_t)pos;
-      if (p.len_mode == 2) v = 8 * p.pool[(int64_t)r * p.pool_blocks + (pos >> 3)] + (int32_t)(pos & 7);
+      if (p.len_mode == 2)
+        v = 8 * (pool_s ? pool_s[pos >> 3] : p.pool[(int64_t)r * p.pool_blocks + (pos >> 3)]) +
+            (int32_t)(pos & 7);
       out[o++] = v;
     }
   }
@@ -665,6 +669,102 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   const int r = blockIdx.y, c = blockIdx.x;
   if (r >= p.num_rows) return;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (p.single) {
+    // Short rows: one CTA holds the row's keys (and, for pool slots, the pool) in shared
+    // memory, compacts the candidates in position order and selects there -- no list in
+    // global memory, no hand-off between CTAs.  The loads go out before the row length is
+    // known; entries at or past it are stale and cleared.
+    if (c != 0) return;
+    constexpr int kPer = kSelSingle / 4 / kSelThreads;    // 16-byte loads per thread
+    uint32_t* keys_s = stage_buf;                          // [kSelSingle]
+    uint32_t* ck = keys_s + kSelSingle;                    // candidates: keys, positions
+    uint32_t* cp = ck + kSelSingle;
+    int32_t* pool_s = reinterpret_cast<int32_t*>(cp + kSelSingle);   // [pool_blocks <= 2048]
+    const uint4* hg = reinterpret_cast<const uint4*>(p.hist + (int64_t)r * kHistBins);
+    const uint4 h0 = hg[tid], h1 = hg[tid + kSelThreads];
+    const uint4* kg = reinterpret_cast<const uint4*>(p.keys + (int64_t)r * p.stride);
+    const int n4 = (int)(p.stride / 4);
+    uint4 kv[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int u = tid + j * kSelThreads;
+      kv[j] = u < n4 ? kg[u] : make_uint4(0, 0, 0, 0);
+    }
+    int len;
+    if (p.len_mode == 2) {
+      // the row covers the active score tiles: 16 valid pool blocks each
+      uint32_t nv = 0;
+      for (int i = tid; i < p.pool_blocks; i += kSelThreads) {
+        const int32_t b = p.pool[(int64_t)r * p.pool_blocks + i];
+        pool_s[i] = b;
+        nv += b >= 0;
+      }
+      nv = block_sum(nv, red);
+      len = min(p.pool_blocks * 8, (int)((nv + 15) / 16) * kTileRows);
+    } else {
+      len = row_len(p, a.seqs, r, red);
+    }
+    len = min(max(len, 0), (int)p.stride);
+    reinterpret_cast<uint4*>(hsm)[tid] = h0;
+    reinterpret_cast<uint4*>(hsm)[tid + kSelThreads] = h1;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int u = tid + j * kSelThreads;
+      uint4 v = kv[j];
+      if (4 * u + 0 >= len) v.x = 0u;
+      if (4 * u + 1 >= len) v.y = 0u;
+      if (4 * u + 2 >= len) v.z = 0u;
+      if (4 * u + 3 >= len) v.w = 0u;
+      if (u < n4) stage_raw[u] = v;
+    }
+    __syncthreads();
+    const Top tp = resolve_top(hsm, (uint32_t)p.k, red);
+    // order-preserving compaction: warp w owns a contiguous run of the row
+    const int run = ((len + 8 * 32 - 1) / (8 * 32)) * 32;
+    const int w_lo = min(len, wid * run), w_hi = min(len, w_lo + run);
+    // (8 keys per lane in flight per step: the loops are latency-bound otherwise)
+    uint32_t cnt = 0;
+    for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
+      uint32_t kk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + 32 * j + lane;
+        kk[j] = i < w_hi ? keys_s[i] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cnt += __popc(__ballot_sync(0xffffffffu, kk[j] != 0u && (kk[j] >> 21) >= tp.b1));
+    }
+    if (lane == 0) wcnt[wid] = cnt;
+    __syncthreads();
+    uint32_t off = 0, n_cand = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+      if (w < wid) off += wcnt[w];
+      n_cand += wcnt[w];
+    }
+    const uint32_t lt = lanemask_lt();
+    for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
+      uint32_t kk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + 32 * j + lane;
+        kk[j] = i < w_hi ? keys_s[i] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const bool pr = kk[j] != 0u && (kk[j] >> 21) >= tp.b1;
+        const uint32_t m = __ballot_sync(0xffffffffu, pr);
+        if (pr) {
+          ck[off + __popc(m & lt)] = kk[j];
+          cp[off + __popc(m & lt)] = (uint32_t)(i0 + 32 * j + lane);
+        }
+        off += __popc(m);
+      }
+    }
+    __syncthreads();
+    StagedSource src{ck, cp, n_cand};
+    final_select(p, r, tp, src, red, hsm, p.len_mode == 2 ? pool_s : nullptr);
+    return;
+  }
   const int len = row_len(p, a.seqs, r, red);
   const int nch = max(1, (len + kSelChunk - 1) / kSelChunk);
   if (c >= nch || c >= p.chunks) return;
@@ -974,6 +1074,7 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
     P.fill = reinterpret_cast<uint32_t*>(wsb + PL.fill);
     P.done = reinterpret_cast<uint32_t*>(wsb + PL.done);
     P.chunks = PL.chunks;
+    P.single = PL.stride <= kSelSingle;
   }
   SelProblem& P = sel.p[0];
   P.k = topk;
@@ -993,7 +1094,10 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
     nprob = 2;
   }
   const dim3 grid(std::max(L.p[0].chunks, nprob == 2 ? L.p[1].chunks : 1), num_q, nprob);
-  const size_t sel_smem = (size_t)2 * kStageCap * 4;
+  // chunked rows: [kStageCap] keys + positions; one-CTA rows: keys, candidate keys and
+  // positions ([kSelSingle] each) and the pool
+  // (one-CTA pool-slot rows have at most kSelSingle / 8 pool blocks)
+  const size_t sel_smem = std::max((size_t)2 * kStageCap * 4, (size_t)(3 * kSelSingle + kSelSingle / 8) * 4);
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sel_smem) != cudaSuccess)
     return CSA2_ERR_CUDA;
