@@ -33,6 +33,10 @@ sys.path.insert(0, ROOT)
 METRIC = "CSA2 decode layer-steps/s at 128K and 1M ctx; achieved HBM GB/s vs roofline"
 UNIT = "layer-steps/s"
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) of one attn_tc_kernel launch at the default workload, from one
+# ncu capture of this kernel (profiles/attn_tc_decoder_step_128k.md); None once the kernel
+# changes
+ATTN_TRAFFIC_BYTES = 448384
 
 
 def peaks():
@@ -321,17 +325,51 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_t = float(t.item())
 
-    # --- roofline of the dominant op: the Full-mode index (score scan + Top-K + pool) ---
+    # --- roofline of the dominant op, sparse attention (attn_tc_kernel + merge): the 20
+    # attention calls of a step (the indices and stash the step left) replayed as one graph,
+    # L2 flushed between replays; per call = time / (replays x 20) ---
+    attn_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+
+        def attn_only():
+            latest, n_idx = dw.indices[0], 1
+            for li, L in enumerate(dw.layers):
+                if L.mode == synth.REINDEX:
+                    latest = dw.indices[n_idx]
+                    n_idx += 1
+                dw.attend(li, latest, stream=stream)
+        attn_only()
+        stream.synchronize()
+        with torch.cuda.graph(attn_graph, stream=stream):
+            attn_only()
+        reps = max(3, min(args.steps, 200))
+        a_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for k in range(-3, reps):
+            flush.zero_()
+            if k >= 0:
+                a_ev[k][0].record(stream)
+            attn_graph.replay()
+            if k >= 0:
+                a_ev[k][1].record(stream)
+    stream.synchronize()
+    attn_s = sum(e[0].elapsed_time(e[1]) for e in a_ev) / 1e3 / (reps * n_layers)
+    del attn_graph
     hbm, tflops, src = peaks()
     n_ctx = W.lengths[0]
+    # per query: the selected FP4 rows (288 B each), the window rows (bf16), Q (bf16) and
+    # the fp32 output
+    attn_bytes = W.num_q * (W.topk * (W.D // 2 + W.D // 16) + W.window * W.D * 2 + W.H * W.D * 2
+                            + W.H * W.D * 4)
+    attn_achieved = attn_bytes / attn_s / 1e9
+    # the Full-mode index (score scan + Top-K + pool), timed inside the steps
     alg_bytes = n_ctx * W.d_I * 2                  # the indexer-K stream, 256 B per entry
     full_s = statistics.mean(full_ms) / 1e3
     achieved = alg_bytes / full_s / 1e9
     steps_total = args.steps * world
     value = steps_total * n_layers / t_total
-    # append 1; each index call: score + select (+ a memset, not a kernel); each
-    # attention: the split kernel, + the merge kernel when split (batch 1 always splits)
-    launches_per_step = (1 if W.append else 0) + 2 * n_index + 2 * n_layers
+    # append 1; each index call: workspace clear + score + select; each attention: the
+    # split kernel, + the merge kernel when split (batch 1 always splits)
+    launches_per_step = (1 if W.append else 0) + 3 * n_index + 2 * n_layers
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
@@ -343,11 +381,18 @@ def run_ours(args, rank, world, local_rank):
                    "window": W.window, "pool": f"{W.pool_blocks}x{W.block}",
                    "l2": "flushed between timed steps (256 MB write)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "csa2_index_full (score scan + Top-K + pool select)",
-                     "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+        "roofline": {"kernel": "csa2_sparse_attn (attn_tc_kernel + merge), one decoder layer",
+                     "bound": "hbm", "achieved": attn_achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": attn_achieved / hbm,
+                     "traffic": ATTN_TRAFFIC_BYTES if W.name == "decoder_step_128k" else None,
+                     "traffic_note": "attn_tc_kernel only (ncu, one launch)",
                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
-                     "alg_bytes_per_launch": alg_bytes, "ms_per_launch": full_s * 1e3},
+                     "alg_bytes_per_launch": attn_bytes, "ms_per_launch": attn_s * 1e3,
+                     "note": "latency-bound at batch 1: 20 CTAs, a chain of dependent phases"},
+        "roofline_index_full": {"kernel": "csa2_index_full (clear + score scan + Top-K + pool select)",
+                                "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                                "frac": achieved / hbm, "alg_bytes_per_launch": alg_bytes,
+                                "ms_per_launch": full_s * 1e3},
         "e2e": {"value": steps_total * n_layers / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
