@@ -245,11 +245,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < HN) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
   if (warp == 0) { tmem_alloc(&ss.tmem_base, G::kTmemCols); tmem_relinquish(); }
   pdl_wait();
-  // Q of the group first, by one thread (heads >= H read as zero: the box runs past the map)
+  // Q of the group first, by one thread (heads >= H read as zero: the box runs past the map),
+  // and a first stash tile, whose address needs nothing from memory
+  const bool stash_first = a.stash != nullptr && a.mode == CSA2_MODE_REUSE && t_begin < t_end &&
+                           t_begin < a.n_idx_tiles;
   if (tid == 0) {
     mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * G::kQChunk);
     for (int c = 0; c < kChunks; ++c)
       tma_load_3d(sQ + c * G::kQChunk, &tm_q, c * 64, h_lo, q, &ss.bar_q);
+    if (stash_first) {
+      mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
+      bulk_g2s(sStage, a.stash + ((int64_t)q * a.n_idx_tiles + t_begin) * G::kStageBytes,
+               G::kStageBytes, &ss.bar_kv);
+    }
   }
   // index of row `tid` of a tile (threads < 128), fetched one tile ahead
   int32_t my_idx = 0;
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
     }
     store_pending = false;
-    if (tid == 0 && from_stash) {            // needs no index: goes out first
+    if (tid == 0 && from_stash && !(t == t_begin && stash_first)) {   // needs no index
       mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
       bulk_g2s(sStage, stile, G::kStageBytes, &ss.bar_kv);
     } else if (tid == 0 && win_tile) {

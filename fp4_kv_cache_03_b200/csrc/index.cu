@@ -719,21 +719,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
     }
     __syncthreads();
     const Top tp = resolve_top(hsm, (uint32_t)p.k, red);
-    // order-preserving compaction: warp w owns a contiguous run of the row
-    const int run = ((len + 8 * 32 - 1) / (8 * 32)) * 32;
+    // order-preserving compaction: warp w owns a contiguous run of the row (a multiple of
+    // 256 keys), lane l takes 8 consecutive keys of each 256 (two 16-byte loads) and
+    // counts locally; a warp prefix sum places every lane's candidates in order
+    const int run = ((len + 8 * 256 - 1) / (8 * 256)) * 256;
     const int w_lo = min(len, wid * run), w_hi = min(len, w_lo + run);
-    // (8 keys per lane in flight per step: the loops are latency-bound otherwise)
+    auto cand_mask = [&](int i0, uint32_t* kk) -> uint32_t {
+      const int i = i0 + 8 * lane;           // (in the array: i + 7 < kSelSingle; past w_hi masked)
+      const uint4 a0 = i < w_hi ? *reinterpret_cast<const uint4*>(keys_s + i) : make_uint4(0, 0, 0, 0);
+      const uint4 a1 = i + 4 < w_hi ? *reinterpret_cast<const uint4*>(keys_s + i + 4) : make_uint4(0, 0, 0, 0);
+      kk[0] = a0.x; kk[1] = a0.y; kk[2] = a0.z; kk[3] = a0.w;
+      kk[4] = a1.x; kk[5] = a1.y; kk[6] = a1.z; kk[7] = a1.w;
+      uint32_t m = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (i + j < w_hi && kk[j] != 0u && (kk[j] >> 21) >= tp.b1) m |= 1u << j;
+      return m;
+    };
     uint32_t cnt = 0;
     for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
       uint32_t kk[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + 32 * j + lane;
-        kk[j] = i < w_hi ? keys_s[i] : 0u;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) cnt += __popc(__ballot_sync(0xffffffffu, kk[j] != 0u && (kk[j] >> 21) >= tp.b1));
+      cnt += __popc(cand_mask(i0, kk));
     }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
     if (lane == 0) wcnt[wid] = cnt;
     __syncthreads();
     uint32_t off = 0, n_cand = 0;
@@ -741,24 +749,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
       if (w < wid) off += wcnt[w];
       n_cand += wcnt[w];
     }
-    const uint32_t lt = lanemask_lt();
     for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
       uint32_t kk[8];
+      const uint32_t m = cand_mask(i0, kk);
+      const uint32_t c = __popc(m);
+      uint32_t incl = c;                     // inclusive prefix over the lanes
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + 32 * j + lane;
-        kk[j] = i < w_hi ? keys_s[i] : 0u;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
+      uint32_t at = off + incl - c;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const bool pr = kk[j] != 0u && (kk[j] >> 21) >= tp.b1;
-        const uint32_t m = __ballot_sync(0xffffffffu, pr);
-        if (pr) {
-          ck[off + __popc(m & lt)] = kk[j];
-          cp[off + __popc(m & lt)] = (uint32_t)(i0 + 32 * j + lane);
+      for (int j = 0; j < 8; ++j)
+        if (m & (1u << j)) {
+          ck[at] = kk[j];
+          cp[at] = (uint32_t)(i0 + 8 * lane + j);
+          ++at;
         }
-        off += __popc(m);
-      }
+      off += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncthreads();
     StagedSource src{ck, cp, n_cand};

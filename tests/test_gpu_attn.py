@@ -43,6 +43,23 @@ def test_short_context_window_and_padding():
     run_attn(W)
 
 
+@pytest.mark.parametrize("D,H", [(256, 40), (512, 12), (128, 64), (256, 1)])
+def test_head_groups_and_dims(D, H):
+    """Every supported D, and head counts that leave a partial 16-head group (the heads past
+    H read as zero); Full then Reuse with the stash, 2 queries of a ragged batch."""
+    W = small_workload(lengths=(700, 3000), D=D, H=H, topk=256, window=128,
+                       modes=("full", "reuse"), outlier_frac=0.01)
+    run_attn(W)
+
+
+def test_many_tiles_per_cta():
+    """More tiles than splits: a CTA loops over several tiles (rescaled running max, the
+    stash stored and loaded per tile) -- 128 queries of one sequence at topk 512."""
+    W = small_workload(lengths=(8192,), q_per_seq=128, D=128, H=16, topk=512, window=128,
+                       modes=("full", "reuse"), q_token0=(8192 - 128,))
+    run_attn(W, queries=[0, 63, 127])
+
+
 def test_window_only_and_empty():
     from fp4_kv_cache_03_b200 import csa2
     dev = "cuda"
