@@ -178,6 +178,27 @@ def oracle_sample(W, budget_s: float):
 
 
 # ----------------------------------------------------------------------------------------
+# the job across ranks: every rank runs an independent replica; the job's time is the
+# slowest rank's, and the job's throughput counts the units of every rank
+# ----------------------------------------------------------------------------------------
+def max_over_ranks(x: float, device="cpu") -> float:
+    """Largest x over all ranks of the default process group (x itself without one)."""
+    import torch
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    dev = "cpu" if dist.get_backend() == "gloo" else device
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(steps_per_rank: int, world: int, layers: int, t_max: float) -> float:
+    """Layer-steps/s of the whole job: every rank's steps over the slowest rank's time."""
+    return steps_per_rank * world * layers / t_max
+
+
+# ----------------------------------------------------------------------------------------
 def run_reference(args, rank):
     """The oracle arm: the same metric, on the host cores, bounded."""
     if rank != 0:
@@ -286,11 +307,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     full_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    t_total = sum(step_ms) / 1e3
-    if world > 1:
-        t = torch.tensor([t_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_total = float(t.item())
+    t_total = max_over_ranks(sum(step_ms) / 1e3, dev)
     st = dw.status()
     if st != csa2.OK:
         raise csa2.CSA2Error(st, "timed steps")
@@ -319,11 +336,7 @@ def run_ours(args, rank, world, local_rank):
                 h.copy_(d, non_blocking=True)
             e2e_ev[k][1].record(stream)
     stream.synchronize()
-    e2e_t = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_t = float(t.item())
+    e2e_t = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, dev)
 
     # --- roofline of the dominant op, sparse attention (attn_tc_kernel + merge): the 20
     # attention calls of a step (the indices and stash the step left) replayed as one graph,
@@ -365,8 +378,7 @@ def run_ours(args, rank, world, local_rank):
     alg_bytes = n_ctx * W.d_I * 2                  # the indexer-K stream, 256 B per entry
     full_s = statistics.mean(full_ms) / 1e3
     achieved = alg_bytes / full_s / 1e9
-    steps_total = args.steps * world
-    value = steps_total * n_layers / t_total
+    value = job_throughput(args.steps, world, n_layers, t_total)
     # append 1; each index call: workspace clear + score + select; each attention: the
     # split kernel, + the merge kernel when split (batch 1 always splits)
     launches_per_step = (1 if W.append else 0) + 3 * n_index + 2 * n_layers
@@ -393,7 +405,8 @@ def run_ours(args, rank, world, local_rank):
                                 "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                                 "frac": achieved / hbm, "alg_bytes_per_launch": alg_bytes,
                                 "ms_per_launch": full_s * 1e3},
-        "e2e": {"value": steps_total * n_layers / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(args.steps, world, n_layers, e2e_t), "unit": UNIT,
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
