@@ -181,6 +181,18 @@ def oracle_sample(W, budget_s: float):
 # the job across ranks: every rank runs an independent replica; the job's time is the
 # slowest rank's, and the job's throughput counts the units of every rank
 # ----------------------------------------------------------------------------------------
+def schedule_of(modes) -> str:
+    """'full, 3 reuse, reindex, 3 reuse, ...': the layer modes, runs of Reuse counted."""
+    out, i = [], 0
+    while i < len(modes):
+        j = i
+        while j < len(modes) and modes[j] == modes[i]:
+            j += 1
+        out.append(modes[i] if j - i == 1 else f"{j - i} {modes[i]}")
+        i = j
+    return ", ".join(out)
+
+
 def max_over_ranks(x: float, device="cpu") -> float:
     """Largest x over all ranks of the default process group (x itself without one)."""
     import torch
@@ -375,7 +387,8 @@ def run_ours(args, rank, world, local_rank):
                             + W.H * W.D * 4)
     attn_achieved = attn_bytes / attn_s / 1e9
     # the Full-mode index (score scan + Top-K + pool), timed inside the steps
-    alg_bytes = n_ctx * W.d_I * 2                  # the indexer-K stream, 256 B per entry
+    # the indexer-K stream, d_I bf16 per visible entry of every query
+    alg_bytes = int(np.sum(W.q_visible())) * W.d_I * 2
     full_s = statistics.mean(full_ms) / 1e3
     achieved = alg_bytes / full_s / 1e9
     value = job_throughput(args.steps, world, n_layers, t_total)
@@ -387,10 +400,13 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp4->fp32",
         "data": "synthetic (seeded; shapes of the pages' decoder, no weights)",
-        "config": {"workload": W.name, "context_entries": n_ctx, "layers": n_layers,
-                   "schedule": "Full+pool, 3 Reuse, 4x(Reindex + 3 Reuse)", "batch": W.num_q,
+        "config": {"workload": W.name,
+                   "context_entries": n_ctx if W.num_seqs == 1 else
+                   f"{W.num_seqs} sequences, {int(np.sum(W.lengths))} in all",
+                   "layers": n_layers, "schedule": schedule_of(W.modes), "batch": W.num_q,
                    "D": W.D, "H": W.H, "indexer": f"{W.H_I}x{W.d_I}", "topk": W.topk,
-                   "window": W.window, "pool": f"{W.pool_blocks}x{W.block}",
+                   "window": W.window,
+                   "pool": f"{W.pool_blocks}x{W.block}" if W.pool_blocks else "none",
                    "l2": "flushed between timed steps (256 MB write)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"kernel": "csa2_sparse_attn (attn_tc_kernel + merge), one decoder layer",

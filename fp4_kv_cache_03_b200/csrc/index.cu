@@ -1104,11 +1104,16 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   }
   const dim3 grid(std::max(L.p[0].chunks, nprob == 2 ? L.p[1].chunks : 1), num_q, nprob);
   // chunked rows: [kStageCap] keys + positions; one-CTA rows: keys, candidate keys and
-  // positions ([kSelSingle] each) and the pool
-  // (one-CTA pool-slot rows have at most kSelSingle / 8 pool blocks)
-  const size_t sel_smem = std::max((size_t)2 * kStageCap * 4, (size_t)(3 * kSelSingle + kSelSingle / 8) * 4);
+  // positions ([kSelSingle] each) and the pool (at most kSelSingle / 8 blocks).  Only a
+  // launch with a one-CTA row asks for the larger size: two chunk CTAs then fit on an SM.
+  bool any_single = sel.p[0].single != 0;
+  if (nprob == 2) any_single = any_single || sel.p[1].single != 0;
+  const size_t sel_smem = any_single ? (size_t)(3 * kSelSingle + kSelSingle / 8) * 4
+                                     : (size_t)2 * kStageCap * 4;
+  // (the function's limit is always the larger size, so that graphs captured with either
+  // launch stay valid)
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sel_smem) != cudaSuccess)
+                           (int)((3 * kSelSingle + kSelSingle / 8) * 4)) != cudaSuccess)
     return CSA2_ERR_CUDA;
   return launch_pdl(select_kernel, grid, dim3(kSelThreads), sel_smem, stream, sel) == cudaSuccess
              ? CSA2_OK
