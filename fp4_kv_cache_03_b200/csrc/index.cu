@@ -161,39 +161,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   if (warp == 1) { tmem_alloc(&ss.tmem_base, a.n_pad * 2 < 32 ? 32 : a.n_pad * 2); tmem_relinquish(); }
   pdl_wait();
 
-  // active tiles of every query, then their exclusive prefix
+  // active tiles of every query, then their exclusive prefix.  Reindex: every query takes
+  // all ceil(pool_blocks / 16) tiles (a pool holds valid blocks first; the slots of -1
+  // blocks get no load and key 0), so the pool is not read here.
   if (kGather) {
-    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = 0;
-    __syncthreads();
-    // (num_q <= 4096 and pool_blocks <= 8192 keep every index below 2^25: 32-bit math)
-    const int n = a.num_q * a.pool_blocks;
-    const int32_t* pl = a.pool + (int64_t)a.q0 * a.pool_blocks;
-    for (int b0 = 0; b0 < n; b0 += 16 * kScoreThreads) {    // 16 loads in flight
-      int32_t v[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int i = b0 + j * kScoreThreads + tid;
-        v[j] = i < n ? __ldg(pl + i) : -1;
-      }
-      // count valid entries per row in a register; one shared atomic per row change
-      int cur_row = -1;
-      uint32_t cnt = 0;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int i = b0 + j * kScoreThreads + tid;
-        if (i >= n) break;
-        const int row = i / a.pool_blocks;
-        if (row != cur_row) {
-          if (cnt) atomicAdd(&rowp[cur_row + 1], cnt);
-          cur_row = row;
-          cnt = 0;
-        }
-        cnt += v[j] >= 0;
-      }
-      if (cnt) atomicAdd(&rowp[cur_row + 1], cnt);
-    }
-    __syncthreads();
-    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = (rowp[i + 1] + 15) / 16;
+    const uint32_t tiles = (uint32_t)((a.pool_blocks + 15) / 16);
+    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles;
   } else {
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles_of<kGather>(a, a.q0 + i);
   }
