@@ -626,12 +626,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // M = max_s m_s and L = sum_s 2^(m_s - M) l_s.  Partials are [head][D] rows, so a thread
 // combines one 4-dim group of one head with 16-byte loads, every load in flight at once.
 constexpr int kMaxSplit = 16;
-__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a, int H, int D) {
+// (small CTAs: at batch 1 the merge's 640 KB of partials spread over 128 SMs)
+constexpr int kMergeThreads = 64;
+__global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const AttnArgs a, int H, int D) {
   pdl_trigger();
   pdl_wait();
   const int q = blockIdx.y, ns = a.nsplit;
   const int n4 = H * D / 4;                  // 4-dim groups of one partial
-  const int g = blockIdx.x * 256 + threadIdx.x;
+  const int g = blockIdx.x * kMergeThreads + threadIdx.x;
   if (g >= n4) return;
   const int h = (g * 4) / D;
   const float4* po = reinterpret_cast<const float4*>(a.part_o + (int64_t)q * ns * H * D) + g;
@@ -765,8 +767,8 @@ cudaError_t launch(AttnArgs a, const uint16_t* q, cudaStream_t st) {
   e = launch_pdl(attn_tc_kernel<D, HN>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
                  (size_t)G::kSmem, st, tm, tm_swa, a);
   if (e != cudaSuccess || a.nsplit <= 1) return e;
-  return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + 255) / 256, a.num_q), dim3(256), 0, st,
-                    a, a.H, D);
+  return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + kMergeThreads - 1) / kMergeThreads, a.num_q),
+                    dim3(kMergeThreads), 0, st, a, a.H, D);
 }
 
 }  // namespace
