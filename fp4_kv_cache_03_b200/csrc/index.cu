@@ -196,7 +196,43 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    if (lane == 0 && t_lo < t_hi) {
+    if (kGather && t_lo < t_hi) {
+      // Reindex: lanes 0-15 each fetch one of the tile's 16 pool blocks (8 rows x 2 halves);
+      // lane 0 waits for the stage, arms its barrier and loads the query
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      int r = find_row(rowp, a.num_q, t_lo);
+      for (uint32_t i = t_lo; i < t_hi; ++i) {
+        if (__shfl_sync(0xffffffffu, *abort, 0)) break;
+        while (rowp[r + 1] <= i) ++r;
+        const int q = a.q0 + r, t = (int)(i - rowp[r]);
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&ss.empty[stage], phase ^ 1, abort, status) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        uint8_t* sa = base + (size_t)stage * stage_bytes;
+        uint8_t* sb = sa + a_bytes;
+        const int64_t row0 = a.seqs.seq_start[q / a.seqs.q_per_seq];
+        const int j = (lane < 16 && t * 16 + lane < a.pool_blocks)
+                          ? __ldg(a.pool + (int64_t)q * a.pool_blocks + t * 16 + lane)
+                          : -1;
+        const uint32_t nvalid = (uint32_t)__popc(__ballot_sync(0xffffffffu, j >= 0));
+        if (lane == 0)
+          mbar_arrive_expect_tx(&ss.full[stage],
+                                (uint32_t)halves * ((uint32_t)a.H_I * 128 + nvalid * 8 * 128));
+        __syncwarp();
+        for (int h = 0; h < halves; ++h) {
+          if (lane == 0) tma_load_2d(sb + h * b_half, &tm_q, h * 64, q * a.H_I, &ss.full[stage]);
+          if (j >= 0)
+            tma_load_2d(sa + h * (kTileRows * 128) + lane * 1024, &tm_k, h * 64,
+                        (int32_t)(row0 + 8 * (int64_t)j), &ss.full[stage]);
+        }
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+    } else if (!kGather && lane == 0 && t_lo < t_hi) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_q);
       int stage = 0;
