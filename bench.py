@@ -36,7 +36,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one attn_tc_kernel launch at the default workload, from one
 # ncu capture of this kernel (profiles/attn_tc_decoder_step_128k.md); None once the kernel
 # changes
-ATTN_TRAFFIC_BYTES = 448384
+ATTN_TRAFFIC_BYTES = 449152
 
 
 def peaks():
