@@ -12,7 +12,8 @@
 //            contiguous, 16-byte pieces) into a staging area -- or, in a Reuse layer with
 //            a stash, come back as one bulk copy of the stage image (with the slots'
 //            validity) that the group's Full / Reindex call stored, so that the layer
-//            reads no indices; window rows go by cp.async straight into the tile;
+//            reads no indices; window rows go straight into the tile, by TMA (one box
+//            per slice) for a tile of window slots only, else by cp.async;
 //   dequant  all 8 warps decode the staged rows to bf16 (exact: a 2-bit-mantissa code times
 //            a 4-bit-mantissa scale) into the KV tile: D/16 slices of [128 keys x 32 B]
 //            with the 32-byte swizzle, which both MMAs read as contiguous 4 KB blocks;

@@ -67,7 +67,8 @@ class DeviceWorkload:
         self.ws_pool = csa2.workspace(csa2.index_pool_workspace(
             nq, max(W.pool_blocks, 1), W.block, W.topk), dev) if self.has_pool else None
         self.ws_attn = csa2.workspace(csa2.sparse_attn_workspace(nq, W.H, W.D, W.topk, W.window), dev)
-        # dequantised selected rows of the latest Full/Reindex layer, for its Reuse layers
+        # staged FP4 rows (codes, scales, validity) of the latest Full/Reindex layer, for
+        # its Reuse layers
         sb = csa2.sparse_attn_stash_bytes(nq, W.D, W.topk)
         self.stash = (torch.empty(sb, dtype=torch.uint8, device=dev)
                       if use_stash and 0 < sb <= self.STASH_LIMIT else None)
