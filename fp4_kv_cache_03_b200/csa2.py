@@ -34,6 +34,23 @@ class Seqs(ctypes.Structure):
                 ("seq_start", c_void_p), ("seq_len", c_void_p)]
 
 
+class Indexer(ctypes.Structure):
+    """csa2_indexer_t: a layer's indexer inputs (FULL / REINDEX)."""
+    _fields_ = [("qI", c_void_p), ("w", c_void_p), ("H_I", c_int32), ("d_I", c_int32),
+                ("idx_k", c_void_p), ("q_visible", c_void_p), ("max_visible", c_int32),
+                ("pool_blocks", c_int32), ("block", c_int32), ("pool", c_void_p),
+                ("workspace", c_void_p), ("ws_bytes", c_size_t)]
+
+
+class Attention(ctypes.Structure):
+    """csa2_attention_t: a layer's attention inputs and outputs."""
+    _fields_ = [("q", c_void_p), ("H", c_int32), ("D", c_int32), ("swa_kv", c_void_p),
+                ("swa_rows", c_int64), ("swa_start", c_void_p), ("q_pos", c_void_p),
+                ("window", c_int32), ("softmax_scale", c_float), ("out", c_void_p),
+                ("lse", c_void_p), ("kv_stash", c_void_p), ("stash_bytes", c_size_t),
+                ("workspace", c_void_p), ("ws_bytes", c_size_t)]
+
+
 _lib = None
 
 _SIGS = {
@@ -58,6 +75,9 @@ _SIGS = {
                                    c_int64, Seqs, c_void_p, c_int32, c_void_p, c_int64, c_void_p,
                                    c_void_p, c_int32, c_float, c_void_p, c_void_p, c_int32,
                                    c_void_p, c_size_t, c_void_p, c_size_t, c_void_p]),
+    "csa2_layer_step": (c_int32, [c_int32, c_int32, c_void_p, c_void_p, c_int64, Seqs, c_int32,
+                                  c_void_p, ctypes.POINTER(Indexer), ctypes.POINTER(Attention),
+                                  c_void_p]),
     "csa2_status_reset": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_fetch": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_string": (ctypes.c_char_p, [c_int32]),
@@ -198,6 +218,30 @@ def sparse_attn(q, kv_codes, kv_scales, seqs: Seqs, indices, swa_kv, swa_start, 
                                   _p(q_pos), window, float(softmax_scale), _p(out), _p(lse),
                                   int(mode), _p(stash), stash.numel() if stash is not None else 0,
                                   _p(ws), ws.numel(), _s(stream)), "csa2_sparse_attn")
+
+
+def layer_step(mode, kv_codes, kv_scales, seqs: Seqs, topk, indices, attn: dict,
+               indexer: dict | None = None, stream=None):
+    """csa2_layer_step: one layer of the schedule.  ``indexer`` (FULL / REINDEX) holds qI, w,
+    idx_k, ws and optionally q_visible, max_visible, pool_blocks, block, pool; ``attn`` holds
+    q, swa_kv, swa_start, q_pos, window, softmax_scale, out, ws and optionally lse, stash."""
+    q = attn["q"]
+    num_q, H, D = q.shape
+    at = Attention(_u16(q), H, D, _u16(attn["swa_kv"]), attn["swa_kv"].shape[0], _p(attn["swa_start"]),
+                   _p(attn["q_pos"]), int(attn["window"]), float(attn["softmax_scale"]),
+                   _p(attn["out"]), _p(attn.get("lse")), _p(attn.get("stash")),
+                   attn["stash"].numel() if attn.get("stash") is not None else 0,
+                   _p(attn["ws"]), attn["ws"].numel())
+    ix = None
+    if indexer is not None:
+        qI = indexer["qI"]
+        ix = Indexer(_u16(qI), _p(indexer["w"]), qI.shape[1], qI.shape[2], _u16(indexer["idx_k"]),
+                     _p(indexer.get("q_visible")), int(indexer.get("max_visible", 0)),
+                     int(indexer.get("pool_blocks", 0)), int(indexer.get("block", 8)),
+                     _p(indexer.get("pool")), _p(indexer["ws"]), indexer["ws"].numel())
+    _check(lib().csa2_layer_step(int(mode), num_q, _p(kv_codes), _p(kv_scales), kv_codes.shape[0],
+                                 seqs, topk, _p(indices), ctypes.byref(ix) if ix is not None else None,
+                                 ctypes.byref(at), _s(stream)), "csa2_layer_step")
 
 
 def status_reset(ws, stream=None) -> None:

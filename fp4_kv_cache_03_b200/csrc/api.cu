@@ -36,3 +36,28 @@ extern "C" int32_t csa2_device_sms(void) {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
   return n;
 }
+
+extern "C" csa2_status_t csa2_layer_step(csa2_mode_t mode, int32_t num_q, const uint8_t* kv_codes,
+                                         const uint8_t* kv_scales, int64_t cap_rows,
+                                         csa2_seqs_t seqs, int32_t topk, int32_t* indices,
+                                         const csa2_indexer_t* ix, const csa2_attention_t* at,
+                                         void* stream) {
+  if (mode != CSA2_MODE_FULL && mode != CSA2_MODE_REINDEX && mode != CSA2_MODE_REUSE)
+    return CSA2_ERR_INVALID_ARG;
+  if (!at || (mode != CSA2_MODE_REUSE && !ix)) return CSA2_ERR_INVALID_ARG;
+  csa2_status_t st = CSA2_OK;
+  if (mode == CSA2_MODE_FULL) {
+    st = csa2_index_full(ix->qI, ix->w, num_q, ix->H_I, ix->d_I, ix->idx_k, cap_rows, seqs,
+                         ix->q_visible, ix->max_visible, topk, indices, ix->pool_blocks,
+                         ix->block, ix->pool, ix->workspace, ix->ws_bytes, stream);
+  } else if (mode == CSA2_MODE_REINDEX) {
+    st = csa2_index_pool(ix->qI, ix->w, num_q, ix->H_I, ix->d_I, ix->idx_k, cap_rows, seqs,
+                         ix->q_visible, ix->pool, ix->pool_blocks, ix->block, topk, indices,
+                         ix->workspace, ix->ws_bytes, stream);
+  }
+  if (st != CSA2_OK) return st;
+  return csa2_sparse_attn(at->q, num_q, at->H, at->D, kv_codes, kv_scales, cap_rows, seqs,
+                          indices, topk, at->swa_kv, at->swa_rows, at->swa_start, at->q_pos,
+                          at->window, at->softmax_scale, at->out, at->lse, mode, at->kv_stash,
+                          at->stash_bytes, at->workspace, at->ws_bytes, stream);
+}

@@ -240,6 +240,54 @@ CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * A layer of the schedule. */
+/* One layer of the CSA2 schedule, driven by its mode ([SURV] §2.2.2 modes table; [MTP]
+ * "CSA2：在层的维度上共享缓存": Full and Reindex layers run their own indexer, Reuse layers
+ * attend with the latest indices):
+ *   FULL     csa2_index_full (building the pool when indexer->pool_blocks > 0) into
+ *            `indices`, then csa2_sparse_attn with mode FULL;
+ *   REINDEX  csa2_index_pool over indexer->pool into `indices`, then csa2_sparse_attn with
+ *            mode REINDEX;
+ *   REUSE    csa2_sparse_attn with mode REUSE and `indices` as given (the latest
+ *            FULL/REINDEX layer's); `indexer` may be NULL.
+ * Every argument keeps the meaning, layout and limits of the call it is passed to; the
+ * two structs only group them.  The first error is returned and nothing after it is
+ * enqueued.  Only host logic: the work is that of the two calls. */
+typedef struct {
+  const uint16_t* qI;        /* device bf16 [num_q][H_I][d_I] */
+  const float* w;            /* device fp32 [num_q][H_I] */
+  int32_t H_I, d_I;
+  const uint16_t* idx_k;     /* device bf16 [cap_rows][d_I] */
+  const int32_t* q_visible;  /* device int32 [num_q] or NULL */
+  int32_t max_visible;       /* FULL: bound on any query's visible entries */
+  int32_t pool_blocks;       /* FULL: 0 = no pool; REINDEX: the pool's blocks per query */
+  int32_t block;             /* pool block size (8) */
+  int32_t* pool;             /* FULL: written when pool_blocks > 0; REINDEX: read */
+  void* workspace;           /* csa2_index_full_workspace / csa2_index_pool_workspace bytes */
+  size_t ws_bytes;
+} csa2_indexer_t;
+typedef struct {
+  const uint16_t* q;         /* device bf16 [num_q][H][D] */
+  int32_t H, D;
+  const uint16_t* swa_kv;    /* device bf16 [swa_rows][D] */
+  int64_t swa_rows;
+  const int64_t* swa_start;  /* device int64 [num_seqs] */
+  const int64_t* q_pos;      /* device int64 [num_q] */
+  int32_t window;
+  float softmax_scale;
+  float* out;                /* device fp32 [num_q][H][D] */
+  float* lse;                /* device fp32 [num_q][H] or NULL */
+  void* kv_stash;            /* or NULL (stateless) */
+  size_t stash_bytes;
+  void* workspace;           /* csa2_sparse_attn_workspace bytes */
+  size_t ws_bytes;
+} csa2_attention_t;
+CSA2_API csa2_status_t csa2_layer_step(csa2_mode_t mode, int32_t num_q, const uint8_t* kv_codes,
+                              const uint8_t* kv_scales, int64_t cap_rows, csa2_seqs_t seqs,
+                              int32_t topk, int32_t* indices, const csa2_indexer_t* indexer,
+                              const csa2_attention_t* attn, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * Status word helpers. */
 /* Enqueue a clear of the status word at the start of `workspace`. */
 CSA2_API csa2_status_t csa2_status_reset(void* workspace, void* stream);

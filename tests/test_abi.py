@@ -108,3 +108,27 @@ def test_device_query_without_gpu_is_harmless(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.csa2_device_sms() == 0
+
+
+def test_host_checks_layer_step(L):
+    """csa2_layer_step rejects a bad mode or missing argument blocks, and passes the
+    first call's host-side status through (nothing is launched on these paths)."""
+    import ctypes as C
+    from fp4_kv_cache_03_b200 import csa2
+    seqs = csa2.Seqs(1, 1, FAKE, FAKE)
+    at = csa2.Attention(FAKE, 16, 128, FAKE, 8, FAKE, FAKE, 4, 0.1, FAKE, None, None, 0, FAKE, 16)
+    ix = csa2.Indexer(FAKE, FAKE, 4, 64, FAKE, None, 4096, 0, 8, None, FAKE, 1 << 30)
+
+    def call(mode, ix_, at_, topk=64):
+        return L.csa2_layer_step(mode, 1, FAKE, FAKE, 100, seqs, topk, FAKE,
+                                 C.byref(ix_) if ix_ is not None else None,
+                                 C.byref(at_) if at_ is not None else None, None)
+    assert call(7, ix, at) == csa2.ERR_INVALID_ARG                    # no such mode
+    assert call(csa2.MODE_REUSE, None, None) == csa2.ERR_INVALID_ARG   # attention args needed
+    assert call(csa2.MODE_FULL, None, at) == csa2.ERR_INVALID_ARG      # Full needs its indexer
+    assert call(csa2.MODE_REINDEX, None, at) == csa2.ERR_INVALID_ARG
+    # Reuse: straight to attention, whose workspace (16 B) is below the status word
+    assert call(csa2.MODE_REUSE, None, at) == csa2.ERR_CAPACITY
+    # Full: the index call's own check comes first (33 indexer heads are unsupported)
+    bad = csa2.Indexer(FAKE, FAKE, 33, 64, FAKE, None, 4096, 0, 8, None, FAKE, 1 << 30)
+    assert call(csa2.MODE_FULL, bad, at) == csa2.ERR_UNSUPPORTED
