@@ -61,16 +61,6 @@ __device__ __forceinline__ int visible_of(const Seqs& s, int q) {
   return v;
 }
 
-// leading pool entries >= 0 (a pool lists ascending block ids, then -1 padding)
-__device__ __forceinline__ int pool_valid(const int32_t* pool_row, int n) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (pool_row[mid] >= 0) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
 // ---------------------------------------------------------------------------------
 // score kernel
 // ---------------------------------------------------------------------------------
@@ -100,9 +90,8 @@ struct ScoreSmem {
   int abort;
 };
 
-template <bool kGather>
-__device__ __forceinline__ int tiles_of(const ScoreArgs& a, int q) {
-  if (kGather) return (pool_valid(a.pool + (int64_t)q * a.pool_blocks, a.pool_blocks) + 15) / 16;
+// Full scan: tiles of query q's visible entries
+__device__ __forceinline__ int full_tiles(const ScoreArgs& a, int q) {
   return (visible_of(a.seqs, q) + kTileRows - 1) / kTileRows;
 }
 
@@ -168,7 +157,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const uint32_t tiles = (uint32_t)((a.pool_blocks + 15) / 16);
     for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles;
   } else {
-    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = tiles_of<kGather>(a, a.q0 + i);
+    for (int i = tid; i < a.num_q; i += kScoreThreads) rowp[i + 1] = full_tiles(a, a.q0 + i);
   }
   __syncthreads();
   if (warp == 0) {
