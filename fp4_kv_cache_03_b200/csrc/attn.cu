@@ -711,16 +711,17 @@ int head_group_of(int num_q, int nsplit, int H) {
   return (int64_t)num_q * nsplit * ((H + 15) / 16) <= sm_count() ? 16 : 32;
 }
 
+// the driver's tensor-map encoder, looked up once (a function-local static: thread-safe)
 PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult qr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
             cudaSuccess &&
         qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
