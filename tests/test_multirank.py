@@ -52,3 +52,28 @@ def test_reference_arm_runs_on_rank_0_only(capsys):
     args = argparse.Namespace(workload="tiny", steps=1, warmup=3, gpus=2)
     bench.run_reference(args, rank=1)                # other ranks exit without work
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line(capsys):
+    """The oracle arm prints one JSON line with the contract's keys, on the host cores."""
+    import argparse
+    import json
+
+    import bench
+    args = argparse.Namespace(workload="tiny", steps=1, warmup=3, gpus=1)
+    bench.run_reference(args, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "layer-steps/s"
+    assert line["metric"] == bench.METRIC and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "layer-steps/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_schedule_description():
+    import bench
+    from fp4_kv_cache_03_b200 import synth
+    assert bench.schedule_of(synth.workload("decoder_step_128k").modes) == \
+        "full, 3 reuse, " + ", ".join(["reindex, 3 reuse"] * 4)
+    assert bench.schedule_of(("full",)) == "full"
