@@ -132,3 +132,18 @@ def test_host_checks_layer_step(L):
     # Full: the index call's own check comes first (33 indexer heads are unsupported)
     bad = csa2.Indexer(FAKE, FAKE, 33, 64, FAKE, None, 4096, 0, 8, None, FAKE, 1 << 30)
     assert call(csa2.MODE_FULL, bad, at) == csa2.ERR_UNSUPPORTED
+
+
+def test_binding_matches_header():
+    """Every entry point of include/csa2.h is bound in csa2.py with as many argument types
+    as the C declaration has parameters (guards the ABI against drift)."""
+    from fp4_kv_cache_03_b200 import csa2
+    text = open(os.path.join(ROOT, "include", "csa2.h"), encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)          # drop comments
+    decls = re.findall(r"CSA2_API[^;(]*?\b(csa2_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S)
+    assert len(decls) >= 12
+    for name, params in decls:
+        assert name in csa2._SIGS, name
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        assert len(csa2._SIGS[name][1]) == n, (name, n, len(csa2._SIGS[name][1]))
