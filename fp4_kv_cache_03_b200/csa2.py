@@ -24,14 +24,15 @@ STATUS_BYTES = 256
 
 class CSA2Error(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = f" [{lib().csa2_last_cuda_error().decode()}]" if status == ERR_CUDA else ""
+        super().__init__(f"{what}: {status_string(status)} (status {status}){detail}")
         self.status = status
 
 
 class Seqs(ctypes.Structure):
     """csa2_seqs_t: ragged batch description (device arrays)."""
     _fields_ = [("num_seqs", c_int32), ("q_per_seq", c_int32),
-                ("seq_start", c_void_p), ("seq_len", c_void_p)]
+                ("seq_start", c_void_p), ("seq_len", c_void_p), ("q_seq", c_void_p)]
 
 
 class Indexer(ctypes.Structure):
@@ -65,6 +66,7 @@ _SIGS = {
     "csa2_index_full_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                           c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p,
                                           c_int32, c_int32, c_void_p, c_void_p]),
+    "csa2_index_full_noalloc_status": (c_int32, [c_void_p]),
     "csa2_index_pool_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32]),
     "csa2_index_pool": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                   c_int64, Seqs, c_void_p, c_void_p, c_int32, c_int32, c_int32,
@@ -81,6 +83,7 @@ _SIGS = {
     "csa2_status_reset": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_fetch": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_string": (ctypes.c_char_p, [c_int32]),
+    "csa2_last_cuda_error": (ctypes.c_char_p, []),
     "csa2_device_sms": (c_int32, []),
 }
 
@@ -130,10 +133,13 @@ def _u16(t):
     return _p(t)
 
 
-def make_seqs(seq_start: torch.Tensor, seq_len: torch.Tensor, q_per_seq: int = 1) -> Seqs:
+def make_seqs(seq_start: torch.Tensor, seq_len: torch.Tensor, q_per_seq: int = 1,
+              q_seq: torch.Tensor | None = None) -> Seqs:
+    """csa2_seqs_t; with ``q_seq`` (int32 [num_q]) each query names its own sequence."""
     assert seq_start.dtype == torch.int64 and seq_len.dtype == torch.int32
-    s = Seqs(int(seq_start.numel()), int(q_per_seq), _p(seq_start), _p(seq_len))
-    s._keep = (seq_start, seq_len)  # keep the tensors alive with the struct
+    assert q_seq is None or q_seq.dtype == torch.int32
+    s = Seqs(int(seq_start.numel()), int(q_per_seq), _p(seq_start), _p(seq_len), _p(q_seq))
+    s._keep = (seq_start, seq_len, q_seq)  # keep the tensors alive with the struct
     return s
 
 
@@ -166,6 +172,7 @@ def index_full(qI, w, idx_k, seqs: Seqs, topk, indices, ws, max_visible, q_visib
                pool_blocks=0, block=8, pool=None, stream=None):
     num_q, H_I, d_I = qI.shape
     assert w.dtype == torch.float32 and indices.dtype == torch.int32
+    assert pool is None or pool.dtype == torch.int32
     _check(lib().csa2_index_full(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
                                  seqs, _p(q_visible), int(max_visible), topk, _p(indices),
                                  pool_blocks, block, _p(pool), _p(ws), ws.numel(), _s(stream)),
@@ -180,10 +187,18 @@ def index_full_noalloc(qI, w, idx_k, seqs: Seqs, topk, indices, max_visible, q_v
     """csa2_index_full with the library's own fixed scratch array instead of a workspace
     (for callers that cannot allocate device memory); see include/csa2.h."""
     num_q, H_I, d_I = qI.shape
+    assert w.dtype == torch.float32 and indices.dtype == torch.int32
+    assert pool is None or pool.dtype == torch.int32
     _check(lib().csa2_index_full_noalloc(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k),
                                          idx_k.shape[0], seqs, _p(q_visible), int(max_visible),
                                          topk, _p(indices), pool_blocks, block, _p(pool),
                                          _s(stream)), "csa2_index_full_noalloc")
+
+
+def index_full_noalloc_status(stream=None) -> int:
+    """Wait for the stream; return the status word of the latest index_full_noalloc call on
+    the current device (0 = OK)."""
+    return int(lib().csa2_index_full_noalloc_status(_s(stream)))
 
 
 def index_pool_workspace(num_q, pool_blocks, block, topk) -> int:
@@ -193,6 +208,7 @@ def index_pool_workspace(num_q, pool_blocks, block, topk) -> int:
 def index_pool(qI, w, idx_k, seqs: Seqs, pool, pool_blocks, block, topk, indices, ws,
                q_visible=None, stream=None):
     num_q, H_I, d_I = qI.shape
+    assert w.dtype == torch.float32 and indices.dtype == torch.int32 and pool.dtype == torch.int32
     _check(lib().csa2_index_pool(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
                                  seqs, _p(q_visible), _p(pool), pool_blocks, block, topk,
                                  _p(indices), _p(ws), ws.numel(), _s(stream)),

@@ -1,6 +1,17 @@
 // Status-word helpers and device queries of the CSA2 C ABI.
 #include "common.cuh"
 
+namespace csa2 {
+namespace {
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+}
+void note_cuda_error(cudaError_t e) { g_last_cuda_error = e; }
+}  // namespace csa2
+
+extern "C" const char* csa2_last_cuda_error(void) {
+  return cudaGetErrorString(csa2::g_last_cuda_error);
+}
+
 extern "C" csa2_status_t csa2_status_reset(void* workspace, void* stream) {
   if (!workspace) return CSA2_ERR_INVALID_ARG;
   return cudaMemsetAsync(workspace, 0, sizeof(int), (cudaStream_t)stream) == cudaSuccess

@@ -5,28 +5,30 @@
 // and window KV; Reuse layers attend with the latest indices) and "FP4 KV 与部署层的几个改动"
 // (E2M1 values with one E4M3 scale per 16 channels).
 //
-// One CTA handles a range of 128-key tiles of one query for one group of 16 or 32 heads
-// (the key slots of a query are [indices[q][0..topk) ; window positions t-W+1 .. t]).
-// Per tile:
-//   stage    the selected rows' FP4 codes and scales are copied with cp.async (row-
-//            contiguous, 16-byte pieces) into a staging area -- or, in a Reuse layer with
-//            a stash, come back as one bulk copy of the stage image (with the slots'
-//            validity) that the group's Full / Reindex call stored, so that the layer
-//            reads no indices; window rows go straight into the tile, by TMA (one box
-//            per slice) for a tile of window slots only, else by cp.async;
-//   dequant  all 8 warps decode the staged rows to bf16 (exact: a 2-bit-mantissa code times
-//            a 4-bit-mantissa scale) into the KV tile: D/16 slices of [128 keys x 32 B]
-//            with the 32-byte swizzle, which both MMAs read as contiguous 4 KB blocks;
-//   S^T      one thread issues tcgen05.mma: S^T[key, head] = KV[key, :] . Q[head, :]
-//            (M = 128 keys, N = the CTA's heads, K = D; Q arrives once by TMA);
-//   softmax  all 8 warps read S^T from TMEM (one key per thread, half the heads per warp),
-//            form per-head maxima and sums with warp reduce-scatters, keep a lazily
-//            rescaled running max per head, and write P (bf16) as [head][key] rows;
-//   O^T      tcgen05.mma: O^T[d, head] += V^T[d, key] . P^T[key, head], reading the same
-//            swizzled KV tile as an MN-major operand (M = 128 dims per slab).
-// The last tile's O^T is normalised and written straight from TMEM; when a query is split
-// over several CTAs they write (m, l, O) partials that a small kernel merges by
-// log-sum-exp.
+// The key slots of a query form 128-slot tiles: ceil(topk / 128) index tiles (the selected
+// cache rows; slots past topk are empty) and ceil(window / 128) window tiles (its window
+// positions t-W+1 .. t).  One CTA takes a contiguous range of one query's tiles with ALL of
+// its heads (N = 16, 32 or 64 in the MMAs): a tcgen05.mma of M = 128 costs about the same
+// for every N <= 64, so one wide instruction replaces four narrow ones and every selected
+// row is gathered and dequantised once.
+//
+// Warp roles (288 threads):
+//   warps 0-7  (256 threads) per index tile: thread (row r, half h) prefetches its half of
+//              row r's FP4 codes and the row's scales into registers one tile ahead (from
+//              the cache, or in a Reuse layer from the stash of the group's Full / Reindex
+//              call), then dequantises them to bf16 (exact: a 2-bit-mantissa code times a
+//              4-bit-mantissa scale) into the KV tile, one 128-dim slab at a time as soon as
+//              the previous tile's O MMA has released that slab; then softmax of the tile
+//              (one key per TMEM lane, half the heads per warp) writes P; at the end, O.
+//   warp 8     one thread: loads Q (TMA, once), the window tiles (TMA, one 16-dim slice per
+//              box, straight into the KV tile) and issues every MMA:
+//                S^T[key, head]  = KV[key, :] . Q[head, :]       (M = 128 keys, K = D)
+//                O^T[d, head]   += V^T[d, key] . P^T[key, head]  (M = 128 dims per slab)
+//              reading the same 32-byte-swizzled KV tile K-major for S^T and MN-major for O^T.
+// The slab barriers let the dequantisation of tile i+1 overlap the O MMAs of tile i, and the
+// S MMAs of tile i+1 start slab by slab.  The last tile's O^T is normalised and written
+// straight from TMEM; when a query is split over several CTAs they write (m, l, O) partials
+// that a small kernel merges by log-sum-exp.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -39,11 +41,13 @@
 namespace csa2 {
 namespace {
 
-constexpr int kThreads = 256;                // 8 warps
-constexpr int kTile = 128;                   // keys per tile (MMA M)
+constexpr int kDqWarps = 8;                  // dequantise / softmax / epilogue warps
+constexpr int kDqThreads = kDqWarps * 32;
+constexpr int kThreads = kDqThreads + 32;    // + the TMA / MMA warp
+constexpr int kTile = 128;                   // key slots per tile (MMA M of S^T)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;         // rescale O only when a max grows by > 2^8
-constexpr int kScaleStride = 48;             // bytes per staged scale row (16-aligned)
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // waits for own copies after an abort
 
 struct AttnArgs {
   int num_q;
@@ -52,7 +56,9 @@ struct AttnArgs {
   int64_t cap_rows;
   const int64_t* seq_start;
   const int32_t* seq_len;
+  const int32_t* q_seq;                      // or null: q / q_per_seq
   int q_per_seq;
+  int num_seqs;
   const int32_t* indices;
   int topk;
   const uint16_t* swa;
@@ -61,12 +67,12 @@ struct AttnArgs {
   const int64_t* q_pos;
   int window;
   int mode;                                  // csa2_mode_t
-  uint8_t* stash;                            // [num_q][n_idx_tiles][stage bytes] or null
-  int n_idx_tiles;                           // tiles holding index slots: ceil(topk / 128)
+  uint8_t* stash;                            // [num_q][n_idx_tiles][stash tile] or null
+  int n_idx_tiles;                           // ceil(topk / 128)
+  int n_win_tiles;                           // ceil(window / 128)
   int H;                                     // real heads
-  int hsplit;                                // head groups (CTAs) per query and split
+  int hsplit;                                // head groups per query (CTAs of HN heads)
   float scale_log2;                          // softmax_scale * log2(e)
-  int n_tiles;                               // tiles of the slot list
   int nsplit, tiles_per_split;
   float* part_o;                             // [num_q][nsplit][H][D]  (nsplit > 1)
   float* part_ml;                            // [num_q][nsplit][H][2]  log2-domain m, l
@@ -75,35 +81,40 @@ struct AttnArgs {
   int* status;
 };
 
+constexpr uint32_t align1024(uint32_t x) { return (x + 1023u) & ~1023u; }
+constexpr uint32_t tmem_cols_for(uint32_t n) {
+  return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
+}
+
 // Shared-memory geometry of one CTA (offsets from a 1024-byte aligned base).
 template <int D, int HN>
 struct Geo {
-  static constexpr int kChunks = D / 64;               // 64-element (128-byte) column chunks
-  static constexpr int kSlabs = D / 128;               // O^T slabs of 128 dims (MMA M)
-  static constexpr uint32_t kQChunk = HN * 128;        // Q chunk: [HN rows][128 B]
+  static constexpr int kSlabs = D / 128;               // 128-dim slabs (O^T MMA M)
+  static constexpr int kChunks = D / 64;               // Q: 64-element (128-byte) chunks
+  static constexpr int kPieces = D / 64;               // 16-byte code pieces per thread
+  static constexpr int kScW = D / 64;                  // 32-bit words of a row's scales
+  static constexpr uint32_t kQChunk = HN * 128;        // [HN rows][128 B]
   // KV tile: D/16 slices of 16 dims, each [128 keys][32 B] with the 32-byte swizzle, so
   // that one MMA K-step (S^T) or one 16-dim chunk of V^T (O^T) is a contiguous 4 KB
   static constexpr uint32_t kKVSlice = kTile * 32;
   static constexpr uint32_t kKVBytes = (D / 16) * kKVSlice;
   static constexpr uint32_t kPChunk = HN * 128;        // P chunk: [HN heads][64 keys]
-  static constexpr uint32_t kCodeStride = D / 2 + 16;  // staged code row (padded: no bank conflicts)
-  static constexpr uint32_t kStageCodes = kTile * kCodeStride;
-  static constexpr uint32_t kStageValid = kStageCodes + kTile * kScaleStride;  // 1 byte per slot
-  static constexpr uint32_t kStageBytes = kStageValid + kTile;
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffKV = (kChunks * kQChunk + 1023) / 1024 * 1024;
+  static constexpr uint32_t kOffKV = align1024(kChunks * kQChunk);
   static constexpr uint32_t kOffP = kOffKV + kKVBytes;
-  static constexpr uint32_t kOffStage = kOffP + (2 * kPChunk + 1023) / 1024 * 1024;
-  static constexpr uint32_t kSmem = 1024 + kOffStage + kStageBytes;
-  // S^T as kSAcc partial accumulators (independent MMA chains), then the O^T slabs
-  static constexpr int kSAcc = 4;
-  static constexpr uint32_t kTmemCols = (kSAcc * HN + kSlabs * HN) <= 128 ? 128 : 256;
-  static_assert(kStageBytes % 16 == 0 && D / 16 <= kScaleStride, "stage layout");
+  static constexpr uint32_t kSmem = 1024 + kOffP + 2 * kPChunk;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(HN * (1 + kSlabs));   // S^T + O^T
+  // one stash tile: codes [128][D/2], scales [128][D/16], validity [128]
+  static constexpr uint32_t kStashCodes = kTile * (D / 2);
+  static constexpr uint32_t kStashValid = kStashCodes + kTile * (D / 16);
+  static constexpr uint32_t kStashBytes = kStashValid + kTile;
+  static_assert(kStashBytes % 16 == 0, "stash tiles stay 16-byte aligned");
 };
 
 template <int HN>
 struct AttnSmem {
-  uint64_t bar_q, bar_s, bar_o, bar_kv;
+  uint64_t bar_q, bar_s, bar_p, bar_o, bar_drain;
+  uint64_t full_dq[4], full_tma[4], empty[4];    // per slab
   uint32_t tmem_base;
   int abort;
   int rescale;
@@ -111,8 +122,8 @@ struct AttnSmem {
   float l_acc[HN];
   float alpha[HN];
   float red[4][HN];
-  int kind[kTile];                           // 0 invalid, 1 FP4 row, 2 window row
-  int64_t src[kTile];                        // cache row (kind 1) or window row (kind 2)
+  int fail;
+  uint8_t valid[2][kTile];                   // slot validity of index tiles k (k even / odd)
 };
 
 // non-negative e4m3 scale byte -> value (bias 7; exponent field 0 is subnormal m * 2^-9)
@@ -192,16 +203,36 @@ __device__ __forceinline__ void warp_reduce_heads(float* v, int lane) {
   }
 }
 
+// N (8, 16 or 32) consecutive TMEM columns of the calling thread's lane, one wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  if constexpr (N == 32) tmem_ld32(taddr, taddr + 16, v);
+  else tmem_ldn<N>(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
+  if constexpr (N == 32) { tmem_st16(taddr, v); tmem_st16(taddr + 16, v + 16); }
+  else tmem_stn<N>(taddr, v);
+}
+
+// the 256 dequantise / softmax threads only (warp 8 never joins)
+__device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// A wait that ignores the abort flag, bounded by kDrainLimitNs: used after an abort for the
+// copies and MMAs this CTA itself has issued, so that none is in flight at exit.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+}
+
 template <int D, int HN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_swa, const AttnArgs a) {
   using G = Geo<D, HN>;
-  constexpr int kChunks = G::kChunks, kSlabs = G::kSlabs;
+  constexpr int kSlabs = G::kSlabs;
   constexpr int HW = HN / 2;                 // heads per warp in softmax and epilogue
-  constexpr int kParts = D / 32;             // 16-byte code pieces (32 values) of a row
-  constexpr int kRowsPerIter = kThreads / kParts;
-  constexpr int kIters = kTile / kRowsPerIter;
   constexpr uint32_t kKVSlice = G::kKVSlice;
   // byte offset of 16-byte unit u (dims 8u .. 8u+7) of key row r in the KV tile
   auto kv_off = [](int r, int u) -> uint32_t {
@@ -217,18 +248,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = base + G::kOffQ;
   uint8_t* sKV = base + G::kOffKV;
   uint8_t* sP = base + G::kOffP;
-  uint8_t* sStage = base + G::kOffStage;
-  uint8_t* sScale = sStage + G::kStageCodes;
-  uint8_t* sValid = sStage + G::kStageValid;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-  const int h0 = (warp >> 2) * HW;           // this warp's heads [h0, h0 + HW) of the group
   const int hg = blockIdx.x % a.hsplit, split = blockIdx.x / a.hsplit, q = blockIdx.y;
-  const int h_lo = hg * HN;                  // first head of the CTA's group
-  const int seq = q / a.q_per_seq;
+  const int h_lo = hg * HN;                  // first head of this CTA's group
   const int t_begin = split * a.tiles_per_split;
-  const int t_end = min(a.n_tiles, t_begin + a.tiles_per_split);
+  const int t_end = min(a.n_idx_tiles + a.n_win_tiles, t_begin + a.tiles_per_split);
+  // processing order: the range's window tiles first (their TMA needs no index), then its
+  // index tiles
+  const int w_lo = max(t_begin, a.n_idx_tiles);
+  const int n_w = max(0, t_end - w_lo);                       // window tiles of the range
+  const int i_hi = min(t_end, a.n_idx_tiles);
+  const int n_i = max(0, i_hi - t_begin);                     // index tiles of the range
+  const int n = n_w + n_i;
   volatile int* abort = &ss.abort;
 
   // set-up that reads no global memory (it overlaps the previous kernel's tail)
@@ -236,382 +268,468 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&ss.bar_q, 1);
     mbar_init(&ss.bar_s, 1);
+    mbar_init(&ss.bar_p, 1);
     mbar_init(&ss.bar_o, 1);
-    mbar_init(&ss.bar_kv, 1);
+    mbar_init(&ss.bar_drain, 1);
+    for (int j = 0; j < 4; ++j) {
+      mbar_init(&ss.full_dq[j], kDqWarps);
+      mbar_init(&ss.full_tma[j], 1);
+      mbar_init(&ss.empty[j], 1);
+    }
     ss.abort = 0;
+    ss.rescale = 0;
     fence_barrier_init();
+  }
+  if (tid == kDqThreads) {
     tma_prefetch_desc(&tm_q);
-    if (a.window > 0 && a.swa_rows > 0) tma_prefetch_desc(&tm_swa);
+    if (a.n_win_tiles > 0 && a.swa_rows > 0) tma_prefetch_desc(&tm_swa);
   }
   if (tid < HN) { ss.m_ref[tid] = -INFINITY; ss.l_acc[tid] = 0.0f; }
   if (warp == 0) { tmem_alloc(&ss.tmem_base, G::kTmemCols); tmem_relinquish(); }
   pdl_wait();
-  // Q of the group first, by one thread (heads >= H read as zero: the box runs past the map),
-  // and a first stash tile, whose address needs nothing from memory
-  const bool stash_first = a.stash != nullptr && a.mode == CSA2_MODE_REUSE && t_begin < t_end &&
-                           t_begin < a.n_idx_tiles;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)kChunks * G::kQChunk);
-    for (int c = 0; c < kChunks; ++c)
-      tma_load_3d(sQ + c * G::kQChunk, &tm_q, c * 64, h_lo, q, &ss.bar_q);
-    if (stash_first) {
-      mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
-      bulk_g2s(sStage, a.stash + ((int64_t)q * a.n_idx_tiles + t_begin) * G::kStageBytes,
-               G::kStageBytes, &ss.bar_kv);
-    }
-  }
-  // index of row `tid` of a tile (threads < 128), fetched one tile ahead
-  int32_t my_idx = 0;
-  auto fetch_idx = [&](int t) {
-    const int slot = t * kTile + tid;
-    const bool stashed = a.stash != nullptr && a.mode == CSA2_MODE_REUSE && t < a.n_idx_tiles;
-    if (tid < kTile && slot < a.topk && !stashed) my_idx = __ldg(a.indices + (int64_t)q * a.topk + slot);
-  };
-  if (t_begin < t_end) fetch_idx(t_begin);
 
-  const int64_t row0 = a.seq_start[seq];
-  const int slen = a.seq_len[seq];
+  // the query's sequence and window (global reads: after the dependency wait)
+  int seq = a.q_seq ? a.q_seq[q] : q / a.q_per_seq;
+  const bool seq_ok = seq >= 0 && seq < a.num_seqs;
+  if (!seq_ok) {
+    if (tid == 0) report(a.status, CSA2_ERR_INVALID_ARG);
+    seq = 0;
+  }
+  const int64_t row0 = seq_ok ? a.seq_start[seq] : 0;
+  const int slen = seq_ok ? a.seq_len[seq] : 0;
   const int64_t t_q = a.q_pos[q];
   const int64_t w0 = t_q - a.window + 1 > 0 ? t_q - a.window + 1 : 0;
-  const int n_win = (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0);
-  const int64_t wrow0 = a.swa_start[seq] + w0;
+  const int n_win = seq_ok ? (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0) : 0;
+  const int64_t wrow0 = (seq_ok && a.window > 0) ? a.swa_start[seq] + w0 : 0;
+
+  // ---- dequantising threads: the FP4 slots this thread loads and converts ----
+  // Warp w covers rows 16w .. 16w+15 of an index tile, as two groups of 8 rows: lane l takes
+  // row 16w + 8g + (l & 7) of group g, and of each 128-dim slab j the 16-byte piece
+  // pq = 4j + (l >> 3) (32 dims).  A warp load then reads 8 rows x 64 contiguous bytes, and a
+  // warp store of one 16-byte unit hits 8 rows x 4 slices, which the 32-byte swizzle spreads
+  // over all banks.
+  const int pl = lane >> 3;                  // piece of the slab (0..3)
+  auto row_of = [&](int g) { return 16 * warp + 8 * g + (lane & 7); };
+  const bool from_stash = a.stash != nullptr && a.mode == CSA2_MODE_REUSE;
+  const bool to_stash = a.stash != nullptr && a.mode != CSA2_MODE_REUSE && hg == 0;
+  uint4 cw[2][kSlabs];                       // codes of (row group, slab)
+  uint32_t sc[2][kSlabs];                    // their two scale bytes (low: first 16 dims)
+  bool vld[2] = {false, false};
+  int32_t nidx[2] = {-1, -1};                // indices of the next tile to fetch
+  auto fetch_index = [&](int t) {
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      const int slot = t * kTile + row_of(g);
+      nidx[g] = (!from_stash && slot < a.topk) ? __ldg(a.indices + (int64_t)q * a.topk + slot) : -1;
+    }
+  };
+  // two scale bytes of row group g, slab j: groups 8j + 2pl, +1 = bytes 2(pl & 1), +1 of
+  // word 2j + (pl >> 1) of the row's scales
+  auto pick_scales = [&](int g, const uint32_t* wv) {
+#pragma unroll
+    for (int j = 0; j < kSlabs; ++j) {
+      const uint32_t w = (pl >> 1) ? wv[2 * j + 1] : wv[2 * j];
+      sc[g][j] = (pl & 1) ? (w >> 16) : (w & 0xFFFFu);
+    }
+  };
+  // Loads index tile t (k-th of the range) into registers and records its slot validity.
+  auto fetch_rows = [&](int t, int k) {
+    if (from_stash) {
+      const uint8_t* st = a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStashBytes;
+      const uint4* sp = reinterpret_cast<const uint4*>(st) + (size_t)warp * (2 * kSlabs) * 32 + lane;
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int j = 0; j < kSlabs; ++j) cw[g][j] = __ldg(sp + (g * kSlabs + j) * 32);
+      const uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (8 * kSlabs / 2);
+      if constexpr (kSlabs == 4) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(ssc));
+        sc[0][0] = v.x & 0xFFFFu; sc[0][1] = v.x >> 16; sc[0][2] = v.y & 0xFFFFu; sc[0][3] = v.y >> 16;
+        sc[1][0] = v.z & 0xFFFFu; sc[1][1] = v.z >> 16; sc[1][2] = v.w & 0xFFFFu; sc[1][3] = v.w >> 16;
+      } else if constexpr (kSlabs == 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(ssc));
+        sc[0][0] = v.x & 0xFFFFu; sc[0][1] = v.x >> 16; sc[1][0] = v.y & 0xFFFFu; sc[1][1] = v.y >> 16;
+      } else {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(ssc));
+        sc[0][0] = v & 0xFFFFu; sc[1][0] = v >> 16;
+      }
+#pragma unroll
+      for (int g = 0; g < 2; ++g) vld[g] = st[G::kStashValid + row_of(g)] != 0;
+    } else {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int r = row_of(g);
+        const int slot = t * kTile + r;
+        const int p = nidx[g];
+        vld[g] = false;
+        if (slot < a.topk) {
+          if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
+            vld[g] = true;
+          } else if (pl == 0 && (p >= slen || p < -1)) {
+            report(a.status, CSA2_ERR_INVALID_ARG);
+          } else if (pl == 0 && p >= 0) {
+            report(a.status, CSA2_ERR_CAPACITY);
+          }
+        }
+        if (vld[g]) {
+          const uint8_t* crow = a.codes + (row0 + p) * (D / 2) + 16 * pl;
+#pragma unroll
+          for (int j = 0; j < kSlabs; ++j) cw[g][j] = __ldg(reinterpret_cast<const uint4*>(crow + 64 * j));
+          const uint8_t* srow = a.scales + (row0 + p) * (D / 16);
+          uint32_t wv[2 * kSlabs];
+          if constexpr (kSlabs >= 2) {
+#pragma unroll
+            for (int c = 0; c < kSlabs / 2; ++c) {
+              const uint4 v = __ldg(reinterpret_cast<const uint4*>(srow) + c);
+              wv[4 * c] = v.x; wv[4 * c + 1] = v.y; wv[4 * c + 2] = v.z; wv[4 * c + 3] = v.w;
+            }
+          } else {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(srow));
+            wv[0] = v.x; wv[1] = v.y;
+          }
+          pick_scales(g, wv);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kSlabs; ++j) { cw[g][j] = make_uint4(0, 0, 0, 0); sc[g][j] = 0u; }
+        }
+      }
+    }
+    if (pl == 0) {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) ss.valid[k & 1][row_of(g)] = vld[g] ? 1 : 0;
+    }
+  };
+  // the first index tile's rows and the index of the one after (their validity is then in
+  // shared memory before the barrier below)
+  if (warp < kDqWarps && n_i > 0) {
+    if (!from_stash) fetch_index(t_begin);
+    fetch_rows(t_begin, 0);
+    if (n_i > 1 && !from_stash) fetch_index(t_begin + 1);
+  }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem_base;
-  const uint32_t tS = tmem;                  // S^T partial a: columns [a HN, (a+1) HN)
-  const uint32_t tO = tmem + G::kSAcc * HN;  // O^T slab j: HN columns from tO + j HN
-  const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+  const uint32_t tS = tmem;                  // S^T: HN columns
+  const uint32_t tO = tmem + HN;             // O^T slab j: HN columns from tO + j HN
 
-  const uint32_t idesc_s = idesc_bf16(kTile, HN);                  // KV, Q both K-major
-  const uint32_t idesc_o = idesc_bf16(kTile, HN, true, false);     // V^T MN-major, P K-major
-  uint32_t ph_s = 0, ph_o = 0, ph_kv = 0;
-  bool q_ready = false, o_init = false, o_pending = false, store_pending = false;
-
-  for (int t = t_begin; t < t_end; ++t) {
-    // Reuse with a stash: the tile's selected rows come back as the stage image that the
-    // Full / Reindex call (head group 0) stored after its gather.
-    const bool stash_tile = a.stash != nullptr && t < a.n_idx_tiles;
-    const bool from_stash = stash_tile && a.mode == CSA2_MODE_REUSE;
-    const bool to_stash = stash_tile && a.mode != CSA2_MODE_REUSE && hg == 0;
-    uint8_t* stile = stash_tile ? a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStageBytes : nullptr;
-    // a tile of window slots only comes in by TMA: D/16 boxes of [128 rows x 16 dims], each
-    // one slice of the tile (rows outside the window are masked, and zeroed below)
-    const bool win_tile = t * kTile >= a.topk;
-    // the previous tile's O^T MMA and stash store must be done before its buffers are rewritten
-    if (store_pending && tid == 0) bulk_wait_read();
-    if (o_pending) {
-      const bool ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status);
-      if (__syncthreads_or(!ok)) break;
-      ph_o ^= 1;
-      o_pending = false;
-      tc_fence_after();
-    } else if (store_pending) {
-      __syncthreads();
-    }
-    store_pending = false;
-    if (tid == 0 && from_stash && !(t == t_begin && stash_first)) {   // needs no index
-      mbar_arrive_expect_tx(&ss.bar_kv, G::kStageBytes);
-      bulk_g2s(sStage, stile, G::kStageBytes, &ss.bar_kv);
-    } else if (tid == 0 && win_tile) {
-      if (a.swa_rows > 0) {
-        // (rows are below 2^31; a start that far outside the map loads zeros only)
-        const int64_t y = wrow0 + ((int64_t)t * kTile - a.topk);
-        const int32_t y0 = (y < -(int64_t)(1 << 30) || y > (int64_t)0x7FFFFF00) ? -(1 << 30) : (int32_t)y;
-        mbar_arrive_expect_tx(&ss.bar_kv, (uint32_t)(D / 16) * kKVSlice);
-        for (int sl = 0; sl < D / 16; ++sl)
-          tma_load_2d(sKV + sl * kKVSlice, &tm_swa, sl * 16, y0, &ss.bar_kv);
-      } else {
-        mbar_arrive(&ss.bar_kv);             // no rows: every slot is masked and zeroed
+  if (warp == kDqWarps) {
+    // =============================== TMA + MMA issue ===============================
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(kTile, HN);                 // KV, Q both K-major
+      const uint32_t idesc_o = idesc_bf16(kTile, HN, true, false);    // V^T MN-major, P K-major
+      const uint64_t kv_desc = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);
+      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t p_desc = sdesc_sw128(smem_u32(sP), 16, 1024);
+      bool ok = true;
+      uint32_t n_dq = 0, n_tma = 0;          // completed phases of full_dq / full_tma
+      int tma_phase = -1, tma_slabs = 0;     // window slabs issued but not yet awaited
+      if (n > 0) {
+        // Q of all heads once (heads >= H read as zero: the box runs past the map)
+        mbar_arrive_expect_tx(&ss.bar_q, (uint32_t)G::kChunks * G::kQChunk);
+        for (int c = 0; c < G::kChunks; ++c)
+          tma_load_3d(sQ + c * G::kQChunk, &tm_q, c * 64, h_lo, q, &ss.bar_q);
       }
-    }
-    // ------------------------- slots -> sources (one thread per row) -------------------------
-    bool ok = true;
-    if (from_stash && tid < kTile) ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
-    if (from_stash) ph_kv ^= 1;
-    if (tid < kTile) {
-      const int slot = t * kTile + tid;
-      int kind = 0;
-      int64_t src = 0;
-      if (slot < a.topk && from_stash) {
-        kind = sValid[tid] ? 1 : 0;              // rows are in the stage already
-      } else if (slot < a.topk) {
-        const int p = my_idx;
-        if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
-          kind = 1;
-          src = row0 + p;
-        } else if (p >= slen || p < -1) {
-          report(a.status, CSA2_ERR_INVALID_ARG);
-        } else if (p >= 0) {
-          report(a.status, CSA2_ERR_CAPACITY);
-        }
-      } else if (slot - a.topk < n_win) {
-        const int64_t grow = wrow0 + (slot - a.topk);
-        if (grow >= 0 && grow < a.swa_rows) {
-          kind = 2;
-          src = grow;
-        } else {
-          report(a.status, CSA2_ERR_CAPACITY);
-        }
-      }
-      ss.kind[tid] = kind;
-      ss.src[tid] = src;
-      if (to_stash && slot < a.topk) sValid[tid] = kind != 0;
-    }
-    if (__syncthreads_or(!ok)) break;
-    if (t + 1 < t_end) fetch_idx(t + 1);
-    // ------------------------- loads (a row's threads are contiguous) -------------------------
-    {
-      const int lp = tid % kParts;
-#pragma unroll
-      for (int it = 0; it < kIters; ++it) {
-        const int r = it * kRowsPerIter + tid / kParts;
-        const int kind = ss.kind[r];
-        if (kind == 1 && !from_stash) {
-          const int64_t grow = ss.src[r];
-          cp_async16(sStage + r * G::kCodeStride + lp * 16, a.codes + grow * (D / 2) + lp * 16);
-          if constexpr (D / 16 >= 16) {
-            if (lp * 16 < D / 16) cp_async16(sScale + r * kScaleStride + lp * 16, a.scales + grow * (D / 16) + lp * 16);
-          } else {
-            if (lp == 0) cp_async8(sScale + r * kScaleStride, a.scales + grow * (D / 16));
+      for (int i = 0; i < n && ok; ++i) {
+        const bool win = i < n_w;
+        if (win) {
+          // window tile: rows straight into the KV tile, one box per 16-dim slice, each slab
+          // once the previous tile's O MMA has released it
+          const int wt = w_lo + i - a.n_idx_tiles;
+          // (rows are below 2^31; a start that far outside the map loads zeros only)
+          const int64_t y = wrow0 + (int64_t)wt * kTile;
+          const int32_t y0 = (y < -(int64_t)(1 << 30) || y > (int64_t)0x7FFFFF00) ? -(1 << 30) : (int32_t)y;
+          tma_phase = (int)n_tma;
+          tma_slabs = 0;
+          for (int j = 0; j < kSlabs && ok; ++j) {
+            if (i > 0) ok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&ss.full_tma[j], 8u * kKVSlice);
+            for (int sl = 0; sl < 8; ++sl)
+              tma_load_2d(sKV + (8 * j + sl) * kKVSlice, &tm_swa, (8 * j + sl) * 16, y0, &ss.full_tma[j]);
+            ++tma_slabs;
           }
-        } else if (kind == 2 && !win_tile) {
-          const uint16_t* src = a.swa + ss.src[r] * D;
+          if (!ok) break;
+        }
+        if (i == 0) ok = mbar_wait(&ss.bar_q, 0, abort, a.status);
+        // S^T = KV . Q^T, slab by slab as the slabs become ready
+        for (int j = 0; j < kSlabs && ok; ++j) {
+          ok = win ? mbar_wait(&ss.full_tma[j], n_tma & 1u, abort, a.status)
+                   : mbar_wait(&ss.full_dq[j], n_dq & 1u, abort, a.status);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int u = 4 * lp + i;
-            cp_async16(sKV + kv_off(r, u), src + u * 8);
-          }
-        } else if (kind == 0 && to_stash && t * kTile + r < a.topk) {
-          // an index slot without a row is stored as zero codes and scales
-          *reinterpret_cast<uint4*>(sStage + r * G::kCodeStride + lp * 16) = make_uint4(0, 0, 0, 0);
-          if (lp * 16 < D / 16) {
-            if constexpr (D / 16 >= 16)
-              *reinterpret_cast<uint4*>(sScale + r * kScaleStride + lp * 16) = make_uint4(0, 0, 0, 0);
-            else
-              *reinterpret_cast<uint2*>(sScale + r * kScaleStride) = make_uint2(0, 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const int k = 8 * j + kk;                                    // 16-dim K-step
+            const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunk + (k & 3) * 32;
+            umma_bf16(tS, kv_desc + (((uint32_t)k * kKVSlice) >> 4), q_desc + (qoff >> 4), idesc_s,
+                      k > 0 ? 1u : 0u);
           }
         }
-      }
-    }
-    cp_async_wait_all();
-    if (win_tile) {
-      ok = mbar_wait(&ss.bar_kv, ph_kv, abort, a.status);
-      ph_kv ^= 1;
-    }
-    if (to_stash) fence_proxy_async_smem();  // staged rows -> the bulk store below
-    if (__syncthreads_or(!ok)) break;
-    if (to_stash) {
-      if (tid == 0) {
-        bulk_s2g(stile, sStage, G::kStageBytes);
-        bulk_commit();
-      }
-      store_pending = true;                  // uniform: every thread takes the same branches
-    }
-    // ------------------------- dequantise into the swizzled tile -------------------------
-    // consecutive threads take consecutive rows: the 8 threads of a quarter warp then store
-    // one 16-byte unit of each of 8 consecutive rows of a slice, which the 32-byte swizzle
-    // spreads over all 32 banks
-    {
-      const int rsub = tid % kRowsPerIter;
-      const int part = tid / kRowsPerIter;
-#pragma unroll
-      for (int it = 0; it < kIters; ++it) {
-        const int r = it * kRowsPerIter + rsub;
-        const int kind = ss.kind[r];
-        // a stash holds zero codes for index slots without a row
-        const bool dec = from_stash ? (t * kTile + r < a.topk) : (kind == 1);
-        if (dec) {
-          const uint4 cw = *reinterpret_cast<const uint4*>(sStage + r * G::kCodeStride + part * 16);
-          const uint32_t sc = *reinterpret_cast<const uint16_t*>(sScale + r * kScaleStride + part * 2);
-          const float s0 = e4m3_val(sc & 0xFFu), s1 = e4m3_val((sc >> 8) & 0xFFu);
-          const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
-          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {              // unit i: 8 values of word w4[i]
-            const uint32_t s2 = i < 2 ? s02 : s12;
-            uint4 o;
-            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-            e2m1x8_to_bf16(w4[i], ow);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ow[k] = mul_bf16x2(ow[k], s2);
-            const int u = 4 * part + i;
-            *reinterpret_cast<uint4*>(sKV + kv_off(r, u)) = o;
-          }
-        } else if (kind == 0) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int u = 4 * part + i;
-            *reinterpret_cast<uint4*>(sKV + kv_off(r, u)) = make_uint4(0, 0, 0, 0);
-          }
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    const int any = __syncthreads_or(tid < kTile && ss.kind[tid] != 0);
-    if (!any) continue;
-
-    // ------------------------------ S^T = KV . Q^T ------------------------------
-    if (tid == 0) {
-      bool okq = true;
-      if (!q_ready) { okq = mbar_wait(&ss.bar_q, 0, abort, a.status); q_ready = okq; }
-      if (okq) {
-        tc_fence_after();
-        const uint64_t kv_desc_k = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);  // KV as K-major A
-        const uint64_t q_desc_k = sdesc_sw128(smem_u32(sQ), 16, 1024);     // Q as K-major B
-        // K-step k accumulates into partial k mod kSAcc: kSAcc independent chains
-#pragma unroll 4
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (uint32_t)k * kKVSlice;
-          const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunk + (k & 3) * 32;
-          umma_bf16(tS + (uint32_t)(k % G::kSAcc) * HN, kv_desc_k + (off >> 4),
-                    q_desc_k + (qoff >> 4), idesc_s, k >= G::kSAcc ? 1u : 0u);
-        }
+        if (!ok) break;
+        if (win) { ++n_tma; tma_phase = -1; } else { ++n_dq; }
         umma_commit(&ss.bar_s);
-      }
-    }
-
-    // ------------------------------ softmax (all 8 warps) ------------------------------
-    // warp w: keys of TMEM lane quadrant (w & 3), heads [h0, h0 + HW)
-    const int r = quad * 32 + lane;               // key row = TMEM lane
-    float v[HW];
-    ok = mbar_wait(&ss.bar_s, ph_s, abort, a.status);
-    ok = __syncthreads_and(ok);
-    ph_s ^= 1;
-    if (!ok) break;
-    tc_fence_after();
-    tmem_ld_sum4<HW>(tS + lane_base + h0, HN, v);   // S^T = the sum of the partials
-    {
-      const bool valid = ss.kind[r] != 0;
-#pragma unroll
-      for (int h = 0; h < HW; ++h) v[h] = valid ? v[h] * a.scale_log2 : -INFINITY;
-      float red[HW];
-#pragma unroll
-      for (int h = 0; h < HW; ++h) red[h] = v[h];
-      warp_reduce_heads<HW, true>(red, lane);     // lane holds head h0 + lane % HW
-      if (lane < HW) ss.red[quad][h0 + lane] = red[0];
-    }
-    if (tid == 0) ss.rescale = 0;
-    __syncthreads();
-    if (tid < HN) {
-      const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
-      ss.alpha[tid] = mt;                          // stash the tile max
-      if (mt > ss.m_ref[tid] + kRescaleLog2) ss.rescale = 1;
-    }
-    __syncthreads();
-    if (ss.rescale) {
-      // move every head's reference max up to its running max; O and l scale by alpha
-      if (tid < HN) {
-        const float mo = ss.m_ref[tid];
-        const float mn = fmaxf(mo, ss.alpha[tid]);
-        const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
-        ss.alpha[tid] = al;
-        ss.l_acc[tid] *= al;
-        ss.m_ref[tid] = mn;
-      }
-      __syncthreads();
-      if (o_init) {
-        float al[HW];
-#pragma unroll
-        for (int i = 0; i < HW; ++i) al[i] = ss.alpha[h0 + i];
-#pragma unroll 1
+        ok = mbar_wait(&ss.bar_p, (uint32_t)i & 1u, abort, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        // O^T += V^T . P^T, slab by slab; each slab is released when its MMAs complete
         for (int j = 0; j < kSlabs; ++j) {
-          float o[HW];
-          const uint32_t ta = tO + lane_base + j * HN + h0;
-          tmem_ldn<HW>(ta, o);
 #pragma unroll
-          for (int i = 0; i < HW; ++i) o[i] *= al[i];
-          tmem_stn<HW>(ta, o);
-        }
-        tmem_wait_st();
-      }
-    }
-    {
-      // p = 2^(s - m_ref), rounded to bf16, written as P[head][key] (a K-major operand:
-      // two 64-key chunks of [HN rows x 128 B], 128-byte swizzle); v becomes the rounded p
-      uint8_t* prow = sP + (r >> 6) * G::kPChunk;
-      const uint32_t unit = (uint32_t)(r & 63) >> 3, byte = (uint32_t)(r & 7) * 2;
-#pragma unroll
-      for (int i = 0; i < HW; ++i) {
-        const int h = h0 + i;
-        const __nv_bfloat16 pb = __float2bfloat16_rn(fast_exp2(v[i] - ss.m_ref[h]));
-        v[i] = __bfloat162float(pb);
-        *reinterpret_cast<__nv_bfloat16*>(prow + h * 128 + ((unit ^ (h & 7)) << 4) + byte) = pb;
-      }
-      warp_reduce_heads<HW, false>(v, lane);
-      if (lane < HW) ss.red[quad][h0 + lane] = v[0];
-      fence_proxy_async_smem();
-      tc_fence_before();
-    }
-    __syncthreads();
-    if (tid < HN) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
-    // ------------------------------ O^T += V^T . P^T ------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint64_t kv_desc_mn = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);    // V^T, MN-major A
-      const uint64_t p_desc_k = sdesc_sw128(smem_u32(sP), 16, 1024);           // P, K-major B
-      // key steps outermost: consecutive MMAs go to the kSlabs independent slabs
-#pragma unroll 2
-      for (int k = 0; k < kTile / 16; ++k) {
-        const uint32_t poff = (uint32_t)(k >> 2) * G::kPChunk + (k & 3) * 32;
-#pragma unroll
-        for (int j = 0; j < kSlabs; ++j) {
-          const uint32_t off = (uint32_t)(8 * j) * kKVSlice + k * 512;   // 16 keys = 2 atoms
-          umma_bf16(tO + j * HN, kv_desc_mn + (off >> 4), p_desc_k + (poff >> 4), idesc_o,
-                    (o_init || k > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t poff = (uint32_t)(kk >> 2) * G::kPChunk + (kk & 3) * 32;
+            const uint32_t off = (uint32_t)(8 * j) * kKVSlice + kk * 512;   // 16 keys = 2 atoms
+            umma_bf16(tO + j * HN, kv_desc + (off >> 4), p_desc + (poff >> 4), idesc_o,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&ss.empty[j]);
         }
       }
-      umma_commit(&ss.bar_o);
-    }
-    o_init = true;
-    o_pending = true;
-  }
-
-  // ------------------------------ epilogue ------------------------------
-  if (store_pending && tid == 0) bulk_wait_read();
-  bool done_ok = !*abort;
-  if (o_pending) done_ok = mbar_wait(&ss.bar_o, ph_o, abort, a.status) && done_ok;
-  done_ok = __syncthreads_and(done_ok);
-  tc_fence_after();
-  const bool partial = a.nsplit > 1;
-  if (done_ok) {
-    // Straight from TMEM: a thread holds one dim of HW heads, so a warp stores one full
-    // 128-byte line per head.  Unsplit: out = O / l.  Split: the unnormalised O (relative
-    // to m_ref) as [H][D] rows of this split, plus (m, l) per head.
-    float* dst = partial ? a.part_o + ((int64_t)q * a.nsplit + split) * Hr * D
-                         : a.out + (int64_t)q * Hr * D;
-    float osc[HW];
-#pragma unroll
-    for (int i = 0; i < HW; ++i) {
-      const float l = ss.l_acc[h0 + i];
-      osc[i] = !o_init ? 0.0f : (partial ? 1.0f : (l > 0.0f ? 1.0f / l : 0.0f));
-    }
-#pragma unroll 1
-    for (int j = 0; j < kSlabs; ++j) {
-      const int d = j * 128 + quad * 32 + lane;
-      float o[HW];
-      if (o_init) {
-        tmem_ldn<HW>(tO + lane_base + j * HN + h0, o);
+      if (ok) {
+        if (n > 0) umma_commit(&ss.bar_o);
       } else {
-#pragma unroll
-        for (int i = 0; i < HW; ++i) o[i] = 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < HW; ++i) {
-        const int h = h_lo + h0 + i;
-        if (h < Hr) dst[h * D + d] = o[i] * osc[i];
+        // abort: the other roles stop waiting; then nothing this thread issued may still be
+        // running at exit (every MMA, the window slabs in flight, Q)
+        *abort = 1;
+        umma_commit(&ss.bar_drain);
+        mbar_drain(&ss.bar_drain, 0);
+        if (tma_phase >= 0)
+          for (int j = 0; j < tma_slabs; ++j) mbar_drain(&ss.full_tma[j], (uint32_t)tma_phase & 1u);
+        if (n > 0) mbar_drain(&ss.bar_q, 0);
       }
     }
-    if (tid < HN && h_lo + tid < Hr) {
-      const int h = h_lo + tid;
-      const float m = ss.m_ref[tid], l = ss.l_acc[tid];
-      if (partial) {
-        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + h) * 2;
-        ml[0] = (o_init && l > 0.0f) ? m : -INFINITY;
-        ml[1] = o_init ? l : 0.0f;
-      } else if (a.lse) {
-        a.lse[(int64_t)q * Hr + h] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+  } else {
+    // ====================== dequantise, softmax, epilogue (warps 0-7) ======================
+    const int qd = warp & 3;                   // TMEM lane quadrant of this warp
+    const int h0 = (warp >> 2) * HW;           // this warp's heads [h0, h0 + HW)
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+
+    // A failed wait (an abort) never leaves the loop early: every thread passes the same
+    // sequence of named barriers, skipping the waits and the MMA hand-offs once failed.
+    bool ok = true;
+    uint32_t ph_s = 0;
+    for (int i = 0; i < n; ++i) {
+      const bool win = i < n_w;
+      const int t = win ? (w_lo + i) : (t_begin + (i - n_w));
+      const int k = i - n_w;                   // index tile number within the range
+      if (!win) {
+        if (to_stash && ok) {
+          // the stash holds the tile in this thread order, so a Reuse layer's loads coalesce
+          uint8_t* st = a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStashBytes;
+          uint4* sp = reinterpret_cast<uint4*>(st) + (size_t)warp * (2 * kSlabs) * 32 + lane;
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int j = 0; j < kSlabs; ++j) sp[(g * kSlabs + j) * 32] = cw[g][j];
+          uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (8 * kSlabs / 2);
+          if constexpr (kSlabs == 4) {
+            *reinterpret_cast<uint4*>(ssc) = make_uint4(sc[0][0] | (sc[0][1] << 16), sc[0][2] | (sc[0][3] << 16),
+                                                        sc[1][0] | (sc[1][1] << 16), sc[1][2] | (sc[1][3] << 16));
+          } else if constexpr (kSlabs == 2) {
+            *reinterpret_cast<uint2*>(ssc) = make_uint2(sc[0][0] | (sc[0][1] << 16), sc[1][0] | (sc[1][1] << 16));
+          } else {
+            *reinterpret_cast<uint32_t*>(ssc) = sc[0][0] | (sc[1][0] << 16);
+          }
+          if (pl == 0) {
+#pragma unroll
+            for (int g = 0; g < 2; ++g) st[G::kStashValid + row_of(g)] = vld[g] ? 1 : 0;
+          }
+        }
+        // dequantise slab by slab into the swizzled tile as the previous tile's O MMA
+        // releases each slab.  The loop is not unrolled (a short body keeps the kernel's
+        // code small: each SM runs it cold); slab j's registers rotate into position 0.
+#pragma unroll 1
+        for (int j = 0; j < kSlabs; ++j) {
+          if (i > 0 && ok) {
+            int wok = 1;
+            if (lane == 0) wok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
+          }
+          if (ok) {
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const uint4 c4 = cw[g][0];
+              const float s0 = e4m3_val(sc[g][0] & 0xFFu), s1 = e4m3_val(sc[g][0] >> 8);
+              const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
+              const uint32_t w4[4] = {c4.x, c4.y, c4.z, c4.w};
+              const int r = row_of(g);
+#pragma unroll
+              for (int u4 = 0; u4 < 4; ++u4) {
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+                e2m1x8_to_bf16(w4[u4], ow);
+                const uint32_t s2 = u4 < 2 ? s02 : s12;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ow[e] = mul_bf16x2(ow[e], s2);
+                *reinterpret_cast<uint4*>(sKV + kv_off(r, 4 * (4 * j + pl) + u4)) = o;
+              }
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0 && ok) mbar_arrive(&ss.full_dq[j]);
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+#pragma unroll
+            for (int jj = 0; jj + 1 < kSlabs; ++jj) { cw[g][jj] = cw[g][jj + 1]; sc[g][jj] = sc[g][jj + 1]; }
+          }
+        }
+        // next index tile: its rows (index already fetched), then the index after it
+        if (ok && k + 1 < n_i) {
+          fetch_rows(t + 1, k + 1);
+          if (k + 2 < n_i && !from_stash) fetch_index(t + 2);
+        }
+      }
+      // ------------------------------ softmax of tile t ------------------------------
+      if (ok) {
+        int wok = 1;
+        if (lane == 0) wok = mbar_wait(&ss.bar_s, ph_s, abort, a.status) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
+      }
+      ph_s ^= 1u;
+      tc_fence_after();
+      const int key = qd * 32 + lane;            // this thread's key row = TMEM lane
+      bool valid;
+      if (win) {
+        const int u = (t - a.n_idx_tiles) * kTile + key;            // window slot
+        const int64_t grow = wrow0 + u;
+        valid = u < n_win && grow >= 0 && grow < a.swa_rows;
+        if (u < n_win && !valid && h0 == 0) report(a.status, CSA2_ERR_CAPACITY);
+      } else {
+        valid = ss.valid[k & 1][key] != 0;       // written a tile ahead, before a barrier
+      }
+      float v[HW];
+      tmem_ld_cols<HW>(tS + lane_base + h0, v);
+      bool over = false;                         // a score above the lazy reference + 2^8
+#pragma unroll
+      for (int e = 0; e < HW; ++e) {
+        v[e] = valid ? v[e] * a.scale_log2 : -INFINITY;
+        over = over || (v[e] > ss.m_ref[h0 + e] + kRescaleLog2);
+      }
+      if (over) ss.rescale = 1;
+      dq_sync();
+      if (ss.rescale) {
+        // the tile's exact per-head max, then every head's reference moves up to its
+        // running max; O and l scale by alpha
+        {
+          float red[HW];
+#pragma unroll
+          for (int e = 0; e < HW; ++e) red[e] = v[e];
+          warp_reduce_heads<HW, true>(red, lane);   // lane holds head h0 + lane % HW
+          if (lane < HW) ss.red[qd][h0 + lane] = red[0];
+        }
+        dq_sync();
+        if (tid < HN) {
+          const float mt = fmaxf(fmaxf(ss.red[0][tid], ss.red[1][tid]), fmaxf(ss.red[2][tid], ss.red[3][tid]));
+          const float mo = ss.m_ref[tid];
+          const float mn = fmaxf(mo, mt);
+          const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+          ss.alpha[tid] = al;
+          ss.l_acc[tid] *= al;
+          ss.m_ref[tid] = mn;
+        }
+        if (tid == 0) ss.rescale = 0;
+        dq_sync();
+        if (i > 0) {   // O holds earlier tiles (their MMAs completed before S of this tile)
+          float al[HW];
+#pragma unroll
+          for (int e = 0; e < HW; ++e) al[e] = ss.alpha[h0 + e];
+#pragma unroll 1
+          for (int j = 0; j < kSlabs; ++j) {
+            float o[HW];
+            const uint32_t ta = tO + lane_base + j * HN + h0;
+            tmem_ld_cols<HW>(ta, o);
+#pragma unroll
+            for (int e = 0; e < HW; ++e) o[e] *= al[e];
+            tmem_st_cols<HW>(ta, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      {
+        // p = 2^(s - m_ref), rounded to bf16, written as P[head][key] (a K-major operand:
+        // two 64-key chunks of [HN rows x 128 B], 128-byte swizzle); v becomes the rounded p.
+        // An empty slot (s = -inf) gives p = 0 even while m_ref is still -inf.
+        uint8_t* prow = sP + (key >> 6) * G::kPChunk;
+        const uint32_t unit = (uint32_t)(key & 63) >> 3, byte = (uint32_t)(key & 7) * 2;
+#pragma unroll
+        for (int e = 0; e < HW; ++e) {
+          const int hh = h0 + e;
+          const float pe = v[e] == -INFINITY ? 0.0f : fast_exp2(v[e] - ss.m_ref[hh]);
+          const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
+          v[e] = __bfloat162float(pb);
+          *reinterpret_cast<__nv_bfloat16*>(prow + hh * 128 + ((unit ^ (hh & 7)) << 4) + byte) = pb;
+        }
+        warp_reduce_heads<HW, false>(v, lane);
+        if (lane < HW) ss.red[qd][h0 + lane] = v[0];
+        fence_proxy_async_smem();
+        tc_fence_before();
+      }
+      dq_sync();
+      if (tid == 0 && ok) mbar_arrive(&ss.bar_p);
+      if (tid < HN) ss.l_acc[tid] += (ss.red[0][tid] + ss.red[1][tid]) + (ss.red[2][tid] + ss.red[3][tid]);
+    }
+
+    // ------------------------------ epilogue ------------------------------
+    bool done_ok = ok && !*abort;
+    if (n > 0 && done_ok) {
+      int wok = 1;
+      if (lane == 0) wok = mbar_wait(&ss.bar_o, 0, abort, a.status) ? 1 : 0;
+      done_ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
+    }
+    // (a vote among the 256 threads: all of them write, or none)
+    if (tid == 0) ss.fail = 0;
+    dq_sync();
+    if (!done_ok) ss.fail = 1;
+    dq_sync();
+    done_ok = ss.fail == 0;
+    tc_fence_after();
+    const bool partial = a.nsplit > 1;
+    if (done_ok) {
+      // O^T from TMEM into shared memory as [head][D] fp32 rows (the KV tile is free: every
+      // MMA has completed), then bulk copies of the H rows.  Unsplit: out = O / l.  Split:
+      // the unnormalised O (relative to m_ref) as this split's [H][D] partial, plus (m, l).
+      float* sO = reinterpret_cast<float*>(sKV);
+      float osc[HW];
+#pragma unroll
+      for (int e = 0; e < HW; ++e) {
+        const float l = ss.l_acc[h0 + e];
+        osc[e] = n == 0 ? 0.0f : (partial ? 1.0f : (l > 0.0f ? 1.0f / l : 0.0f));
+      }
+#pragma unroll 1
+      for (int j = 0; j < kSlabs; ++j) {
+        const int d = j * 128 + qd * 32 + lane;
+        float o[HW];
+        if (n > 0) {
+          tmem_ld_cols<HW>(tO + lane_base + j * HN + h0, o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < HW; ++e) o[e] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < HW; ++e) sO[(h0 + e) * D + d] = o[e] * osc[e];
+      }
+      fence_proxy_async_smem();
+      dq_sync();
+      float* dst = partial ? a.part_o + ((int64_t)q * a.nsplit + split) * Hr * D
+                           : a.out + (int64_t)q * Hr * D;
+      const int n_h = min(HN, Hr - h_lo);        // real heads of this group
+      if (tid < 32) {
+        for (int hh = tid; hh < n_h; hh += 32)
+          bulk_s2g(dst + (size_t)(h_lo + hh) * D, sO + (size_t)hh * D, D * 4);
+        bulk_commit();
+        bulk_wait_all();
+      }
+      if (tid >= 32 && tid < 32 + n_h) {
+        const int hh = tid - 32;
+        const float m = ss.m_ref[hh], l = ss.l_acc[hh];
+        if (partial) {
+          float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + h_lo + hh) * 2;
+          ml[0] = (n > 0 && l > 0.0f) ? m : -INFINITY;
+          ml[1] = n > 0 ? l : 0.0f;
+        } else if (a.lse) {
+          a.lse[(int64_t)q * Hr + h_lo + hh] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
       }
     }
   }
@@ -627,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // M = max_s m_s and L = sum_s 2^(m_s - M) l_s.  Partials are [head][D] rows, so a thread
 // combines one 4-dim group of one head with 16-byte loads, every load in flight at once.
 constexpr int kMaxSplit = 16;
-// (small CTAs: at batch 1 the merge's 640 KB of partials spread over 128 SMs)
+// (small CTAs: at batch 1 the merge's partials spread over many SMs)
 constexpr int kMergeThreads = 64;
 __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const AttnArgs a, int H, int D) {
   pdl_trigger();
@@ -677,20 +795,8 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const AttnArg
 // ---------------------------------------------------------------------------------
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int n_tiles_of(int topk, int window) { return (topk + window + kTile - 1) / kTile; }
-
-int nsplit_of(int num_q, int n_tiles) {
-  if (n_tiles <= 1) return 1;
-  return std::max(1, std::min(std::min(n_tiles, kMaxSplit), 512 / std::max(1, num_q)));
-}
-
-bool attn_shape_ok(int H, int D) {
-  return H >= 1 && H <= 64 && (D == 128 || D == 256 || D == 512);
-}
-
-// bytes of one staged tile (and of one stash tile): padded code rows, scale rows, then one
-// validity byte per slot
-size_t stage_bytes_of(int D) { return (size_t)kTile * ((size_t)D / 2 + 16 + kScaleStride + 1); }
+int idx_tiles_of(int topk) { return (topk + kTile - 1) / kTile; }
+int win_tiles_of(int window) { return (window + kTile - 1) / kTile; }
 
 int sm_count() {
   static std::atomic<int> cached[64];
@@ -705,11 +811,19 @@ int sm_count() {
   return n;
 }
 
-// Heads per CTA: groups of 16 while every CTA of the call fits on the GPU at once (the
-// latency-bound small batches), else 32 (fewer repeated gathers per query).
-int head_group_of(int num_q, int nsplit, int H) {
-  return (int64_t)num_q * nsplit * ((H + 15) / 16) <= sm_count() ? 16 : 32;
+// Key splits per query: enough CTAs to cover the SMs when the batch is small (each split
+// adds a partial of H x D fp32 that the merge reads back), one split from a full wave on.
+int nsplit_of(int num_q, int n_tiles) {
+  if (n_tiles <= 1 || num_q <= 0) return 1;
+  const int per_q = std::max(1, sm_count() / num_q);
+  return std::max(1, std::min(std::min(n_tiles, kMaxSplit), per_q));
 }
+
+bool attn_shape_ok(int H, int D) {
+  return H >= 1 && H <= 64 && (D == 128 || D == 256 || D == 512);
+}
+
+size_t stash_tile_bytes(int D) { return (size_t)kTile * ((size_t)D / 2 + (size_t)D / 16 + 1); }
 
 // the driver's tensor-map encoder, looked up once (a function-local static: thread-safe)
 PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
@@ -725,8 +839,8 @@ PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
   return fn;
 }
 
-// Q as a [num_q][H][D] bf16 map with boxes of 64 dims x HN heads: heads >= H of the last
-// group fall outside the map and read as zero.
+// Q as a [num_q][H][D] bf16 map with boxes of 64 dims x HN heads: heads >= H fall outside
+// the map and read as zero.
 bool make_q_map(CUtensorMap* tm, const uint16_t* q, int num_q, int H, int D, int HN) {
   auto fn = attn_encode_fn();
   if (!fn) return false;
@@ -757,20 +871,40 @@ template <int D, int HN>
 cudaError_t launch(AttnArgs a, const uint16_t* q, cudaStream_t st) {
   using G = Geo<D, HN>;
   CUtensorMap tm;
-  if (!make_q_map(&tm, q, a.num_q, a.H, D, HN)) return cudaErrorInvalidValue;
+  if (!make_q_map(&tm, q, a.num_q, a.H, D, HN)) return checked(cudaErrorInvalidValue);
   CUtensorMap tm_swa;
-  std::memset(&tm_swa, 0, sizeof(tm_swa));  // not read without window slots
-  if (a.window > 0 && a.swa_rows > 0 && !make_swa_map(&tm_swa, a.swa, a.swa_rows, D))
-    return cudaErrorInvalidValue;
-  a.hsplit = (a.H + HN - 1) / HN;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, HN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem);
+  std::memset(&tm_swa, 0, sizeof(tm_swa));  // not read without window tiles
+  if (a.n_win_tiles > 0 && a.swa_rows > 0 && !make_swa_map(&tm_swa, a.swa, a.swa_rows, D))
+    return checked(cudaErrorInvalidValue);
+  cudaError_t e = checked(cudaFuncSetAttribute(attn_tc_kernel<D, HN>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem));
   if (e != cudaSuccess) return e;
   e = launch_pdl(attn_tc_kernel<D, HN>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
                  (size_t)G::kSmem, st, tm, tm_swa, a);
   if (e != cudaSuccess || a.nsplit <= 1) return e;
   return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + kMergeThreads - 1) / kMergeThreads, a.num_q),
                     dim3(kMergeThreads), 0, st, a, a.H, D);
+}
+
+// Heads per CTA.  Every CTA gathers and dequantises its query's tiles once for all of its
+// heads, and an MMA costs about the same for N = 16 as for N = 64; but a CTA's softmax,
+// output and split partial scale with its heads.  Small batches that leave SMs idle split
+// the heads into groups of 16 (or 32); from a full wave on, one CTA takes all heads.
+int heads_per_cta(int num_q, int nsplit, int H) {
+  const int64_t ctas = (int64_t)num_q * nsplit;
+  if (ctas * ((H + 15) / 16) <= sm_count()) return 16;
+  if (ctas * ((H + 31) / 32) <= sm_count()) return 32;
+  return 64;
+}
+
+template <int D>
+cudaError_t launch_d(AttnArgs a, const uint16_t* q, cudaStream_t st) {
+  const int all = a.H <= 16 ? 16 : a.H <= 32 ? 32 : 64;     // one group of all heads
+  const int g = std::min(heads_per_cta(a.num_q, a.nsplit, a.H), all);
+  a.hsplit = (a.H + g - 1) / g;
+  if (g == 16) return launch<D, 16>(a, q, st);
+  if (g == 32) return launch<D, 32>(a, q, st);
+  return launch<D, 64>(a, q, st);
 }
 
 }  // namespace
@@ -780,13 +914,13 @@ using namespace csa2;
 
 extern "C" size_t csa2_sparse_attn_stash_bytes(int32_t num_q, int32_t D, int32_t topk) {
   if (num_q < 0 || D < 1 || topk < 0) return 0;
-  return (size_t)num_q * ((topk + kTile - 1) / kTile) * stage_bytes_of(D);
+  return (size_t)num_q * idx_tiles_of(topk) * stash_tile_bytes(D);
 }
 
 extern "C" size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
                                              int32_t window) {
   if (num_q < 0 || H < 1 || D < 1 || topk < 0 || window < 0) return 0;
-  const int ns = nsplit_of(num_q, n_tiles_of(topk, window));
+  const int ns = nsplit_of(num_q, idx_tiles_of(topk) + win_tiles_of(window));
   size_t off = CSA2_STATUS_BYTES;
   if (ns > 1) {
     off = a256(off + (size_t)num_q * ns * H * D * 4);
@@ -807,16 +941,15 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
                                           void* stream) {
   if (num_q < 0 || topk < 0 || topk > 2048 || window < 0 || window > 1024) return CSA2_ERR_INVALID_ARG;
   if (!attn_shape_ok(H, D)) return CSA2_ERR_UNSUPPORTED;
-  if (seqs.num_seqs < 1 || seqs.q_per_seq < 1 || (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)
+  if (seqs.num_seqs < 1 ||
+      (!seqs.q_seq && (seqs.q_per_seq < 1 || (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)))
     return CSA2_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < csa2_sparse_attn_workspace(num_q, H, D, topk, window))
     return CSA2_ERR_CAPACITY;
   if (mode != CSA2_MODE_FULL && mode != CSA2_MODE_REINDEX && mode != CSA2_MODE_REUSE)
     return CSA2_ERR_INVALID_ARG;
-  if (kv_stash && (stash_bytes < csa2_sparse_attn_stash_bytes(num_q, D, topk) ||
-                   (reinterpret_cast<uintptr_t>(kv_stash) & 15)))
-    return kv_stash && (reinterpret_cast<uintptr_t>(kv_stash) & 15) ? CSA2_ERR_INVALID_ARG
-                                                                    : CSA2_ERR_CAPACITY;
+  if (kv_stash && (reinterpret_cast<uintptr_t>(kv_stash) & 15)) return CSA2_ERR_INVALID_ARG;
+  if (kv_stash && stash_bytes < csa2_sparse_attn_stash_bytes(num_q, D, topk)) return CSA2_ERR_CAPACITY;
   if (num_q == 0) return CSA2_OK;
   if (num_q > 65535) return CSA2_ERR_UNSUPPORTED;       // queries are a grid dimension
   if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
@@ -830,18 +963,22 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   AttnArgs a{};
   a.num_q = num_q;
   a.codes = kv_codes; a.scales = kv_scales; a.cap_rows = cap_rows;
-  a.seq_start = seqs.seq_start; a.seq_len = seqs.seq_len; a.q_per_seq = seqs.q_per_seq;
+  a.seq_start = seqs.seq_start; a.seq_len = seqs.seq_len;
+  a.q_seq = seqs.q_seq; a.q_per_seq = seqs.q_per_seq > 0 ? seqs.q_per_seq : 1;
+  a.num_seqs = seqs.num_seqs;
   a.indices = indices; a.topk = topk;
   a.swa = swa_kv; a.swa_rows = swa_rows; a.swa_start = swa_start; a.q_pos = q_pos;
   a.window = window;
   a.mode = (int)mode;
   a.stash = static_cast<uint8_t*>(kv_stash);
-  a.n_idx_tiles = (topk + kTile - 1) / kTile;
+  a.n_idx_tiles = idx_tiles_of(topk);
+  a.n_win_tiles = (swa_rows > 0) ? win_tiles_of(window) : 0;
   a.H = H;
   a.scale_log2 = softmax_scale * kLog2e;
-  a.n_tiles = n_tiles_of(topk, window);
-  a.nsplit = nsplit_of(num_q, a.n_tiles);
-  a.tiles_per_split = (a.n_tiles + a.nsplit - 1) / a.nsplit;
+  const int n_tiles = a.n_idx_tiles + a.n_win_tiles;
+  // (the split count depends on the call's shape only, as the workspace size does)
+  a.nsplit = nsplit_of(num_q, idx_tiles_of(topk) + win_tiles_of(window));
+  a.tiles_per_split = std::max(1, (n_tiles + a.nsplit - 1) / a.nsplit);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
   size_t off = CSA2_STATUS_BYTES;
@@ -851,10 +988,9 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   a.out = out; a.lse = lse;
 
   cudaStream_t st = (cudaStream_t)stream;
-  const bool g16 = head_group_of(num_q, a.nsplit, H) == 16;
   cudaError_t e = cudaSuccess;
-  if (D == 128) e = g16 ? launch<128, 16>(a, q, st) : launch<128, 32>(a, q, st);
-  else if (D == 256) e = g16 ? launch<256, 16>(a, q, st) : launch<256, 32>(a, q, st);
-  else e = g16 ? launch<512, 16>(a, q, st) : launch<512, 32>(a, q, st);
+  if (D == 128) e = launch_d<128>(a, q, st);
+  else if (D == 256) e = launch_d<256>(a, q, st);
+  else e = launch_d<512>(a, q, st);
   return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

@@ -38,6 +38,14 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The CUDA runtime error of the latest failed call this host thread made into the library
+// (cudaSuccess if none); csa2_last_cuda_error() returns its message.
+void note_cuda_error(cudaError_t e);
+inline cudaError_t checked(cudaError_t e) {
+  if (e != cudaSuccess) note_cuda_error(e);
+  return e;
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args&&... args) {
@@ -51,7 +59,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  return checked(cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...));
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -157,6 +165,10 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // wait until every committed shared -> global bulk copy has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until every committed shared -> global bulk copy has completed (writes performed)
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------

@@ -46,13 +46,28 @@ struct Seqs {
   const int64_t* seq_start;
   const int32_t* seq_len;
   const int32_t* q_visible;
+  const int32_t* q_seq;            // or null: q / q_per_seq
   int q_per_seq;
+  int num_seqs;
   int max_visible;
   int* status;
 };
 
+// the sequence of query q, or -1 for an out-of-range q_seq value
+__device__ __forceinline__ int seq_of(const Seqs& s, int q) {
+  const int seq = s.q_seq ? s.q_seq[q] : q / s.q_per_seq;
+  return (seq >= 0 && seq < s.num_seqs) ? seq : -1;
+}
+
+// first cache row of query q's sequence (0 for an invalid sequence, which sees nothing)
+__device__ __forceinline__ int64_t row0_of(const Seqs& s, int q) {
+  const int seq = seq_of(s, q);
+  return seq >= 0 ? s.seq_start[seq] : 0;
+}
+
 __device__ __forceinline__ int visible_of(const Seqs& s, int q) {
-  const int seq = q / s.q_per_seq;
+  const int seq = seq_of(s, q);
+  if (seq < 0) { report(s.status, CSA2_ERR_INVALID_ARG); return 0; }
   const int len = s.seq_len[seq];
   int v = s.q_visible ? s.q_visible[q] : len;
   if (v < 0) { report(s.status, CSA2_ERR_INVALID_ARG); v = 0; }
@@ -204,7 +219,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
-        const int64_t row0 = a.seqs.seq_start[q / a.seqs.q_per_seq];
+        const int64_t row0 = row0_of(a.seqs, q);
         const int j = (lane < 16 && t * 16 + lane < a.pool_blocks)
                           ? __ldg(a.pool + (int64_t)q * a.pool_blocks + t * 16 + lane)
                           : -1;
@@ -233,7 +248,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (!mbar_wait(&ss.empty[stage], phase ^ 1, abort, status)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
-        const int64_t row0 = a.seqs.seq_start[q / a.seqs.q_per_seq];
+        const int64_t row0 = row0_of(a.seqs, q);
         uint32_t bytes = (uint32_t)halves * (uint32_t)a.H_I * 128;
         int32_t blk_row[16];
         if (kGather) {
@@ -1014,7 +1029,8 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   if (ws_bytes < L.total) return CSA2_ERR_CAPACITY;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(wsb);
-  Seqs sq{seqs.seq_start, seqs.seq_len, q_visible, seqs.q_per_seq, max_visible, status};
+  Seqs sq{seqs.seq_start, seqs.seq_len, q_visible, seqs.q_seq,
+          seqs.q_per_seq > 0 ? seqs.q_per_seq : 1, seqs.num_seqs, max_visible, status};
 
   {
     const uint32_t n16 = (uint32_t)((L.zero_hi - L.zero_lo) / 16);   // both ends 256-aligned
@@ -1057,7 +1073,7 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
     // at least one tile per CTA on average for the largest plausible work
     const int64_t tiles_bound = (int64_t)sa.num_q * ((row_len + kTileRows - 1) / kTileRows);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_bound));
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (checked(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
       return CSA2_ERR_CUDA;
     if (launch_pdl(kern, dim3(grid), dim3(kScoreThreads), smem, stream, tm_k, tm_q, sa) !=
@@ -1111,8 +1127,8 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
                                      : (size_t)2 * kStageCap * 4;
   // (the function's limit is always the larger size, so that graphs captured with either
   // launch stay valid)
-  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)((3 * kSelSingle + kSelSingle / 8) * 4)) != cudaSuccess)
+  if (checked(cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)((3 * kSelSingle + kSelSingle / 8) * 4))) != cudaSuccess)
     return CSA2_ERR_CUDA;
   return launch_pdl(select_kernel, grid, dim3(kSelThreads), sel_smem, stream, sel) == cudaSuccess
              ? CSA2_OK
@@ -1121,20 +1137,33 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
 
 csa2_status_t check_common(const uint16_t* qI, const float* w, int num_q, int H_I, int d_I,
                            const uint16_t* idx_k, int64_t cap_rows, const csa2_seqs_t& seqs,
-                           int topk, const int32_t* indices, const void* ws) {
+                           int topk, const int32_t* indices) {
   if (num_q < 0 || num_q > 65535 || H_I < 1 || H_I > 32 || (d_I != 64 && d_I != 128))
     return CSA2_ERR_UNSUPPORTED;
   if (topk < 1 || topk > 4096) return CSA2_ERR_UNSUPPORTED;
   if (cap_rows <= 0 || cap_rows > 0x7FFFFFFF) return CSA2_ERR_INVALID_ARG;
-  if (seqs.num_seqs < 1 || seqs.q_per_seq < 1 ||
-      (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)
+  if (seqs.num_seqs < 1 ||
+      (!seqs.q_seq && (seqs.q_per_seq < 1 || (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)))
     return CSA2_ERR_INVALID_ARG;
   if (num_q == 0) return CSA2_OK;
-  if (!qI || !w || !idx_k || !indices || !seqs.seq_start || !seqs.seq_len || !ws)
+  if (!qI || !w || !idx_k || !indices || !seqs.seq_start || !seqs.seq_len)
     return CSA2_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(qI) & 15) || (reinterpret_cast<uintptr_t>(idx_k) & 15) ||
-      (reinterpret_cast<uintptr_t>(ws) & 255))
+  if ((reinterpret_cast<uintptr_t>(qI) & 15) || (reinterpret_cast<uintptr_t>(idx_k) & 15))
     return CSA2_ERR_INVALID_ARG;
+  return CSA2_OK;
+}
+
+csa2_status_t check_ws(const void* ws) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return CSA2_ERR_INVALID_ARG;
+  return CSA2_OK;
+}
+
+// the Full-mode arguments beyond those of check_common; adjusts `block` when there is no pool
+csa2_status_t check_full(int max_visible, int pool_blocks, int& block, const int32_t* pool) {
+  if (max_visible < 0) return CSA2_ERR_INVALID_ARG;
+  if (pool_blocks < 0 || pool_blocks > 8192) return CSA2_ERR_UNSUPPORTED;
+  if (pool_blocks > 0 && (!pool || !pow2_le32(block))) return CSA2_ERR_UNSUPPORTED;
+  if (pool_blocks == 0) block = 8;
   return CSA2_OK;
 }
 
@@ -1163,13 +1192,10 @@ extern "C" csa2_status_t csa2_index_full(const uint16_t* qI, const float* w, int
                                          int32_t topk, int32_t* indices, int32_t pool_blocks,
                                          int32_t block, int32_t* pool, void* workspace,
                                          size_t ws_bytes, void* stream) {
-  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices,
-                                  workspace);
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices);
   if (st != CSA2_OK || num_q == 0) return st;
-  if (max_visible < 0) return CSA2_ERR_INVALID_ARG;
-  if (pool_blocks < 0 || pool_blocks > 8192) return CSA2_ERR_UNSUPPORTED;
-  if (pool_blocks > 0 && (!pool || !pow2_le32(block))) return CSA2_ERR_UNSUPPORTED;
-  if (pool_blocks == 0) block = 8;
+  if ((st = check_ws(workspace)) != CSA2_OK) return st;
+  if ((st = check_full(max_visible, pool_blocks, block, pool)) != CSA2_OK) return st;
   return run_index<false>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, max_visible,
                           topk, indices, pool_blocks, block, pool, nullptr, workspace, ws_bytes,
                           (cudaStream_t)stream);
@@ -1182,9 +1208,9 @@ extern "C" csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int
                                          int32_t pool_blocks, int32_t block, int32_t topk,
                                          int32_t* indices, void* workspace, size_t ws_bytes,
                                          void* stream) {
-  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices,
-                                  workspace);
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices);
   if (st != CSA2_OK || num_q == 0) return st;
+  if ((st = check_ws(workspace)) != CSA2_OK) return st;
   if (block != 8 || pool_blocks < 1 || pool_blocks > 8192 || !pool) return CSA2_ERR_UNSUPPORTED;
   // positions inside the pool are bounded by the pool; the visibility bound only clamps
   // q_visible values that exceed the sequence
@@ -1228,21 +1254,24 @@ extern "C" csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float
                                                  int32_t max_visible, int32_t topk,
                                                  int32_t* indices, int32_t pool_blocks,
                                                  int32_t block, int32_t* pool, void* stream) {
-  if (max_visible < 0) return CSA2_ERR_INVALID_ARG;
-  if (pool_blocks < 0 || pool_blocks > 8192) return CSA2_ERR_UNSUPPORTED;
-  const size_t need = csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks,
-                                                pool_blocks > 0 ? block : 8);
+  // the same argument checks, in the same order, as csa2_index_full; the size check last
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices);
+  if (st != CSA2_OK || num_q == 0) return st;
+  if ((st = check_full(max_visible, pool_blocks, block, pool)) != CSA2_OK) return st;
+  const size_t need = csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks, block);
   if (need == 0 || need > (size_t)CSA2_INDEX_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_CAPACITY;
   void* ws = index_scratch_address();
   if (!ws) return CSA2_ERR_CUDA;
-  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices, ws);
-  if (st != CSA2_OK || num_q == 0) return st;
-  if (pool_blocks > 0 && (!pool || !pow2_le32(block))) return CSA2_ERR_UNSUPPORTED;
-  if (pool_blocks == 0) block = 8;
   // the status word starts clear on every call (the histograms are cleared by run_index)
   if (cudaMemsetAsync(ws, 0, CSA2_STATUS_BYTES, (cudaStream_t)stream) != cudaSuccess)
     return CSA2_ERR_CUDA;
   return run_index<false>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, max_visible,
                           topk, indices, pool_blocks, block, pool, nullptr, ws,
                           (size_t)CSA2_INDEX_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
+}
+
+extern "C" csa2_status_t csa2_index_full_noalloc_status(void* stream) {
+  void* ws = index_scratch_address();
+  if (!ws) return CSA2_ERR_CUDA;
+  return csa2_status_fetch(ws, stream);
 }

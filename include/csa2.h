@@ -75,12 +75,17 @@ typedef enum {
 
 #define CSA2_STATUS_BYTES 256
 
-/* Ragged batch description.  Query q belongs to sequence q / q_per_seq. */
+/* Ragged batch description, shared by every call.
+ * Query q belongs to sequence q_seq[q] when q_seq is not NULL (any mix of decode queries
+ * and chunks of several queries per sequence; a value outside [0, num_seqs) makes that
+ * query see nothing and records CSA2_ERR_INVALID_ARG), else to sequence q / q_per_seq, in
+ * which case num_seqs * q_per_seq must equal num_q. */
 typedef struct {
   int32_t num_seqs;           /* host: number of sequences (>= 1) */
-  int32_t q_per_seq;          /* host: queries per sequence (decode: 1) */
+  int32_t q_per_seq;          /* host: queries per sequence when q_seq is NULL (decode: 1) */
   const int64_t* seq_start;   /* device [num_seqs]: cache row of position 0 */
   const int32_t* seq_len;     /* device [num_seqs]: entries stored for the sequence */
+  const int32_t* q_seq;       /* device [num_q] or NULL: the sequence of every query */
 } csa2_seqs_t;
 
 /* ---------------------------------------------------------------------------------
@@ -152,12 +157,18 @@ CSA2_API csa2_status_t csa2_index_full(const uint16_t* qI, const float* w, int32
  *     exceeds CSA2_INDEX_NOALLOC_SCRATCH_BYTES the call returns CSA2_ERR_CAPACITY and
  *     enqueues nothing (8 MiB covers one query over 1,048,576 entries with a pool).
  *   - Set-up: the first call on a device looks up the array's device address (with that
- *     device current) and caches it; make that first call before any stream capture.
+ *     device current) and caches it; make that first call before any stream capture.  A
+ *     cudaDeviceReset() invalidates the cached address: do not call this entry point on a
+ *     device after resetting it in the same process.
  *   - Sharing: every call on a device uses the same array and leaves its contents there;
  *     each call clears what must start at zero.  Calls that overlap on the GPU (different
  *     streams, or different host threads) race on the array: serialise them.
- *   - Device-side value errors are handled as in csa2_index_full (skipped / clamped) but
- *     cannot be fetched: the status word lives in the library's array. */
+ *   - Arguments are checked in the same order and with the same status codes as
+ *     csa2_index_full; the size limit is checked after them.
+ *   - Device-side value errors are handled as in csa2_index_full (skipped / clamped) and
+ *     recorded in the array's own status word, which each call clears when it starts:
+ *     csa2_index_full_noalloc_status() returns it for the latest call on the current
+ *     device. */
 #define CSA2_INDEX_NOALLOC_SCRATCH_BYTES (8u << 20)
 CSA2_API csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float* w, int32_t num_q,
                                                int32_t H_I, int32_t d_I, const uint16_t* idx_k,
@@ -166,6 +177,9 @@ CSA2_API csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float* 
                                                int32_t topk, int32_t* indices,
                                                int32_t pool_blocks, int32_t block, int32_t* pool,
                                                void* stream);
+/* Wait for `stream`, then return the status word of the latest csa2_index_full_noalloc call
+ * on the current device (CSA2_OK if its kernels recorded no error). */
+CSA2_API csa2_status_t csa2_index_full_noalloc_status(void* stream);
 
 /* ---------------------------------------------------------------------------------
  * a5. Reindex over the pool ([SURV] §2.2.2: Reindex reuses main KV and indexer K but has
@@ -296,6 +310,9 @@ CSA2_API csa2_status_t csa2_status_reset(void* workspace, void* stream);
 CSA2_API csa2_status_t csa2_status_fetch(const void* workspace, void* stream);
 /* Static text for a status code. */
 CSA2_API const char* csa2_status_string(csa2_status_t status);
+/* The CUDA runtime's message for the latest CUDA failure (a call that returned
+ * CSA2_ERR_CUDA) made by the calling host thread, or "no error".  Static storage. */
+CSA2_API const char* csa2_last_cuda_error(void);
 /* Number of streaming multiprocessors of the current device (0 on error). */
 CSA2_API int32_t csa2_device_sms(void);
 

@@ -98,9 +98,15 @@ def test_host_checks_attention(L):
     assert call(mode=7) == csa2.ERR_INVALID_ARG
     assert call(stash=ctypes.c_void_p(0x200000), stash_bytes=16) == csa2.ERR_CAPACITY
     assert call(stash=ctypes.c_void_p(0x200008), stash_bytes=1 << 30) == csa2.ERR_INVALID_ARG
-    # 4 tiles of 128 staged rows: padded codes (256 + 16 B), a 48-byte scale row and a
-    # validity byte
-    assert L.csa2_sparse_attn_stash_bytes(1, 512, 512) == 4 * 128 * (256 + 16 + 48 + 1)
+    # 4 tiles of 128 rows: codes (256 B), scales (32 B) and a validity byte per row
+    assert L.csa2_sparse_attn_stash_bytes(1, 512, 512) == 4 * 128 * (256 + 32 + 1)
+    # a per-query sequence map lifts the num_seqs x q_per_seq = num_q rule
+    bad = csa2.Seqs(2, 1, FAKE, FAKE)                       # 2 x 1 != 1 query
+    mapped = csa2.Seqs(2, 0, FAKE, FAKE, FAKE)             # q_seq given: q_per_seq unused
+    args = lambda seqs: (FAKE, 1, 16, 128, FAKE, FAKE, 100, seqs, FAKE, 64, FAKE, 100, FAKE, FAKE,
+                         128, 0.1, FAKE, None, 0, None, 0, ctypes.c_void_p(0x100000), 300, None)
+    assert L.csa2_sparse_attn(*args(bad)) == csa2.ERR_INVALID_ARG
+    assert L.csa2_sparse_attn(*args(mapped)) == csa2.ERR_CAPACITY   # passes the map check
 
 
 def test_device_query_without_gpu_is_harmless(L):

@@ -130,3 +130,12 @@ def test_reuse_stash_equals_stateless():
     for li in range(len(W.modes)):
         assert torch.equal(a.out[li], b.out[li]), li
         assert torch.equal(a.lse[li], b.lse[li]), li
+
+
+def test_all_heads_in_one_cta():
+    """A batch large enough that one CTA takes all 64 heads of a query (N = 64 in the MMAs),
+    with the stash in the staging order of that path."""
+    W = small_workload(lengths=(6000,), q_per_seq=80, D=512, H=64, H_I=16, d_I=128, topk=256,
+                       window=128, modes=("full", "reuse"), q_token0=(6000 - 80,),
+                       outlier_frac=0.01)
+    run_attn(W, queries=[0, 41, 79])

@@ -29,6 +29,7 @@ def _both(dw, L, W):
                             pool=got_pool)
     torch.cuda.synchronize()
     assert csa2.status_fetch(dw.ws_full) == csa2.OK
+    assert csa2.index_full_noalloc_status() == csa2.OK     # the array's own status word
     return ref_idx, ref_pool, got_idx, got_pool
 
 
@@ -67,3 +68,25 @@ def test_noalloc_rejects_sizes_beyond_its_array():
         csa2.index_full_noalloc(L.qI, L.w, dw.idx_k, dw.seqs, W.topk, idx, 4_000_000)
     assert e.value.status == csa2.ERR_CAPACITY
     assert csa2.index_full_workspace(1, 4_000_000, W.topk) > csa2.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_argument_errors_match_the_workspace_entry_point():
+    """Bad arguments give the same status as csa2_index_full, before the size check."""
+    from fp4_kv_cache_03_b200 import csa2
+    from fp4_kv_cache_03_b200.workload import DeviceWorkload
+    W = small_workload(lengths=(4096,), modes=("full",), seed=24)
+    dw = DeviceWorkload(W)
+    L = dw.layers[0]
+    idx = torch.zeros(1, 64, dtype=torch.int32, device="cuda")
+    for topk, pool_blocks, block in ((0, 0, 8), (5000, 0, 8), (64, 16, 3), (64, 9000, 8)):
+        codes = []
+        for fn in (lambda: csa2.index_full(L.qI, L.w, dw.idx_k, dw.seqs, topk, idx, dw.ws_full,
+                                           4_000_000, pool_blocks=pool_blocks, block=block,
+                                           pool=idx if pool_blocks else None),
+                   lambda: csa2.index_full_noalloc(L.qI, L.w, dw.idx_k, dw.seqs, topk, idx,
+                                                   4_000_000, pool_blocks=pool_blocks,
+                                                   block=block, pool=idx if pool_blocks else None)):
+            with pytest.raises(csa2.CSA2Error) as e:
+                fn()
+            codes.append(e.value.status)
+        assert codes[0] == codes[1] == csa2.ERR_UNSUPPORTED, (topk, pool_blocks, block, codes)
