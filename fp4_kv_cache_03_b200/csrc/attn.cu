@@ -288,19 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) { tmem_alloc(&ss.tmem_base, G::kTmemCols); tmem_relinquish(); }
   pdl_wait();
 
-  // the query's sequence and window (global reads: after the dependency wait)
-  int seq = a.q_seq ? a.q_seq[q] : q / a.q_per_seq;
-  const bool seq_ok = seq >= 0 && seq < a.num_seqs;
-  if (!seq_ok) {
-    if (tid == 0) report(a.status, CSA2_ERR_INVALID_ARG);
-    seq = 0;
-  }
-  const int64_t row0 = seq_ok ? a.seq_start[seq] : 0;
-  const int slen = seq_ok ? a.seq_len[seq] : 0;
-  const int64_t t_q = a.q_pos[q];
-  const int64_t w0 = t_q - a.window + 1 > 0 ? t_q - a.window + 1 : 0;
-  const int n_win = seq_ok ? (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0) : 0;
-  const int64_t wrow0 = (seq_ok && a.window > 0) ? a.swa_start[seq] + w0 : 0;
+  // the query's sequence and window: read after the dependency wait, below, once the first
+  // tile's index (or stash) loads are in flight
+  int64_t row0 = 0, wrow0 = 0;
+  int slen = 0, n_win = 0;
 
   // ---- dequantising threads: the FP4 slots this thread loads and converts ----
   // Warp w covers rows 16w .. 16w+15 of an index tile, as two groups of 8 rows: lane l takes
@@ -399,12 +390,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < 2; ++g) ss.valid[k & 1][row_of(g)] = vld[g] ? 1 : 0;
     }
   };
-  // the first index tile's rows and the index of the one after (their validity is then in
-  // shared memory before the barrier below)
-  if (warp < kDqWarps && n_i > 0) {
-    if (!from_stash) fetch_index(t_begin);
+  // The first index tile's index (or stash rows) goes out first; then the sequence lookups;
+  // then the first tile's rows and the index of the one after (their validity is then in
+  // shared memory before the barrier below).
+  const bool first_fetch = warp < kDqWarps && n_i > 0;
+  if (first_fetch) {
+    if (from_stash) fetch_rows(t_begin, 0);
+    else fetch_index(t_begin);
+  }
+  {
+    int seq = a.q_seq ? a.q_seq[q] : q / a.q_per_seq;
+    const bool seq_ok = seq >= 0 && seq < a.num_seqs;
+    if (!seq_ok) {
+      if (tid == 0) report(a.status, CSA2_ERR_INVALID_ARG);
+      seq = 0;
+    }
+    row0 = seq_ok ? a.seq_start[seq] : 0;
+    slen = seq_ok ? a.seq_len[seq] : 0;
+    const int64_t t_q = a.q_pos[q];
+    const int64_t w0 = t_q - a.window + 1 > 0 ? t_q - a.window + 1 : 0;
+    n_win = seq_ok ? (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0) : 0;
+    wrow0 = (seq_ok && a.window > 0) ? a.swa_start[seq] + w0 : 0;
+  }
+  if (first_fetch && !from_stash) {
     fetch_rows(t_begin, 0);
-    if (n_i > 1 && !from_stash) fetch_index(t_begin + 1);
+    if (n_i > 1) fetch_index(t_begin + 1);
   }
 
   tc_fence_before();
