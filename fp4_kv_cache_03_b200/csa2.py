@@ -85,6 +85,7 @@ _SIGS = {
     "csa2_status_string": (ctypes.c_char_p, [c_int32]),
     "csa2_last_cuda_error": (ctypes.c_char_p, []),
     "csa2_device_sms": (c_int32, []),
+    "csa2_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
 }
 
 
@@ -267,6 +268,12 @@ def status_reset(ws, stream=None) -> None:
 def status_fetch(ws, stream=None) -> int:
     """Wait for the stream; return the status word recorded in ``ws`` (0 = OK)."""
     return int(lib().csa2_status_fetch(_p(ws), _s(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Bound of the kernels' waits for later launches (0 = the default 2 s); returns the
+    previous bound."""
+    return int(lib().csa2_set_wait_limit_ns(int(ns)))
 
 
 def device_sms() -> int:

@@ -1,12 +1,20 @@
 // Status-word helpers and device queries of the CSA2 C ABI.
 #include "common.cuh"
 
+#include <atomic>
+
 namespace csa2 {
 namespace {
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+std::atomic<uint64_t> g_wait_ns{kWaitLimitNs};
 }
 void note_cuda_error(cudaError_t e) { g_last_cuda_error = e; }
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 }  // namespace csa2
+
+extern "C" uint64_t csa2_set_wait_limit_ns(uint64_t ns) {
+  return csa2::g_wait_ns.exchange(ns == 0 ? csa2::kWaitLimitNs : ns, std::memory_order_relaxed);
+}
 
 extern "C" const char* csa2_last_cuda_error(void) {
   return cudaGetErrorString(csa2::g_last_cuda_error);

@@ -47,7 +47,6 @@ constexpr int kThreads = kDqThreads + 32;    // + the TMA / MMA warp
 constexpr int kTile = 128;                   // key slots per tile (MMA M of S^T)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;         // rescale O only when a max grows by > 2^8
-constexpr uint64_t kDrainLimitNs = 200000000ull;   // waits for own copies after an abort
 
 struct AttnArgs {
   int num_q;
@@ -79,6 +78,7 @@ struct AttnArgs {
   float* out;
   float* lse;
   int* status;
+  uint64_t wait_ns;                          // bound of every wait
 };
 
 constexpr uint32_t align1024(uint32_t x) { return (x + 1023u) & ~1023u; }
@@ -217,14 +217,6 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
 
 // the 256 dequantise / softmax threads only (warp 8 never joins)
 __device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-// A wait that ignores the abort flag, bounded by kDrainLimitNs: used after an abort for the
-// copies and MMAs this CTA itself has issued, so that none is in flight at exit.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
-}
 
 template <int D, int HN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -453,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_phase = (int)n_tma;
           tma_slabs = 0;
           for (int j = 0; j < kSlabs && ok; ++j) {
-            if (i > 0) ok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status);
+            if (i > 0) ok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status, a.wait_ns);
             if (!ok) break;
             mbar_arrive_expect_tx(&ss.full_tma[j], 8u * kKVSlice);
             for (int sl = 0; sl < 8; ++sl)
@@ -462,11 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
         }
-        if (i == 0) ok = mbar_wait(&ss.bar_q, 0, abort, a.status);
+        if (i == 0) ok = mbar_wait(&ss.bar_q, 0, abort, a.status, a.wait_ns);
         // S^T = KV . Q^T, slab by slab as the slabs become ready
         for (int j = 0; j < kSlabs && ok; ++j) {
-          ok = win ? mbar_wait(&ss.full_tma[j], n_tma & 1u, abort, a.status)
-                   : mbar_wait(&ss.full_dq[j], n_dq & 1u, abort, a.status);
+          ok = win ? mbar_wait(&ss.full_tma[j], n_tma & 1u, abort, a.status, a.wait_ns)
+                   : mbar_wait(&ss.full_dq[j], n_dq & 1u, abort, a.status, a.wait_ns);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -480,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (win) { ++n_tma; tma_phase = -1; } else { ++n_dq; }
         umma_commit(&ss.bar_s);
-        ok = mbar_wait(&ss.bar_p, (uint32_t)i & 1u, abort, a.status);
+        ok = mbar_wait(&ss.bar_p, (uint32_t)i & 1u, abort, a.status, a.wait_ns);
         if (!ok) break;
         tc_fence_after();
         // O^T += V^T . P^T, slab by slab; each slab is released when its MMAs complete
@@ -552,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < kSlabs; ++j) {
           if (i > 0 && ok) {
             int wok = 1;
-            if (lane == 0) wok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status) ? 1 : 0;
+            if (lane == 0) wok = mbar_wait(&ss.empty[j], (uint32_t)(i - 1) & 1u, abort, a.status, a.wait_ns) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
           }
           if (ok) {
@@ -593,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------ softmax of tile t ------------------------------
       if (ok) {
         int wok = 1;
-        if (lane == 0) wok = mbar_wait(&ss.bar_s, ph_s, abort, a.status) ? 1 : 0;
+        if (lane == 0) wok = mbar_wait(&ss.bar_s, ph_s, abort, a.status, a.wait_ns) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
       }
       ph_s ^= 1u;
@@ -684,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool done_ok = ok && !*abort;
     if (n > 0 && done_ok) {
       int wok = 1;
-      if (lane == 0) wok = mbar_wait(&ss.bar_o, 0, abort, a.status) ? 1 : 0;
+      if (lane == 0) wok = mbar_wait(&ss.bar_o, 0, abort, a.status, a.wait_ns) ? 1 : 0;
       done_ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
     }
     // (a vote among the 256 threads: all of them write, or none)
@@ -996,6 +988,7 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   off = a256(off + (size_t)num_q * a.nsplit * H * D * 4);
   a.part_ml = reinterpret_cast<float*>(ws + off);
   a.out = out; a.lse = lse;
+  a.wait_ns = wait_limit_ns();
 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;

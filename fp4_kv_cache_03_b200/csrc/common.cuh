@@ -17,8 +17,11 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
-// every spin in this library gives up after this many nanoseconds of %globaltimer
+// every spin in this library gives up after this many nanoseconds of %globaltimer (the
+// default; csa2_set_wait_limit_ns() changes it for later launches)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// the limit the next launch passes to its kernels (host side)
+uint64_t wait_limit_ns();
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -103,21 +106,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase of `bar` with the given parity has completed.  Gives up when
-// `*abort` becomes non-zero (another role gave up) or after kWaitLimitNs; in the
-// latter case it raises `*abort` and records CSA2_ERR_TIMEOUT.  Returns true on success.
+// `*abort` becomes non-zero (another role gave up) or after `limit_ns`; in the latter case
+// it raises `*abort` and records CSA2_ERR_TIMEOUT.  Returns true on success.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       report(status, CSA2_ERR_TIMEOUT);
       return false;
     }
   }
+}
+
+// A wait for a phase of this CTA's own copies or MMAs after an abort: it ignores the abort
+// flag (those operations complete by themselves) and gives up after 200 ms.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > 200000000ull) return;
 }
 
 // ---------------------------------------------------------------------------------

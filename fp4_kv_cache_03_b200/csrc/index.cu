@@ -94,6 +94,7 @@ struct ScoreArgs {
   int block;                       // block size for bkeys (power of two <= 32)
   uint32_t* hist;                  // [q][kHistBins] first-digit histogram of keys
   uint32_t* bhist;                 // same for block keys (or null)
+  uint64_t wait_ns;                // bound of every wait
 };
 
 struct ScoreSmem {
@@ -101,6 +102,7 @@ struct ScoreSmem {
   uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     rowp[0] = 0;
     for (int s = 0; s < S; ++s) { mbar_init(&ss.full[s], 1); mbar_init(&ss.empty[s], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&ss.tfull[i], 1); mbar_init(&ss.tempty[i], 4); }
+    mbar_init(&ss.drain, 1);
     ss.abort = 0;
     fence_barrier_init();
   }
@@ -209,13 +212,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t filled = 0;                     // stages holding a load (bit s), its parity below
+      uint32_t filled_parity = 0;
       int r = find_row(rowp, a.num_q, t_lo);
       for (uint32_t i = t_lo; i < t_hi; ++i) {
         if (__shfl_sync(0xffffffffu, *abort, 0)) break;
         while (rowp[r + 1] <= i) ++r;
         const int q = a.q0 + r, t = (int)(i - rowp[r]);
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(&ss.empty[stage], phase ^ 1, abort, status) ? 1 : 0;
+        if (lane == 0) ok = mbar_wait(&ss.empty[stage], phase ^ 1, abort, status, a.wait_ns) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
@@ -234,18 +239,26 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             tma_load_2d(sa + h * (kTileRows * 128) + lane * 1024, &tm_k, h * 64,
                         (int32_t)(row0 + 8 * (int64_t)j), &ss.full[stage]);
         }
+        filled |= 1u << stage;
+        filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
+      // no load of this CTA may still be landing when it exits (after an abort the MMA warp
+      // has not consumed every stage); a consumed stage's phase has completed already
+      if (lane == 0)
+        for (int st = 0; st < S; ++st)
+          if (filled & (1u << st)) mbar_drain(&ss.full[st], (filled_parity >> st) & 1u);
     } else if (!kGather && lane == 0 && t_lo < t_hi) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_q);
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t filled = 0, filled_parity = 0;  // as in the Reindex producer
       int r = find_row(rowp, a.num_q, t_lo);
       for (uint32_t i = t_lo; i < t_hi && !*abort; ++i) {
         while (rowp[r + 1] <= i) ++r;
         const int q = a.q0 + r, t = (int)(i - rowp[r]);
-        if (!mbar_wait(&ss.empty[stage], phase ^ 1, abort, status)) break;
+        if (!mbar_wait(&ss.empty[stage], phase ^ 1, abort, status, a.wait_ns)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
         const int64_t row0 = row0_of(a.seqs, q);
@@ -274,8 +287,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         (int32_t)(row0 + (int64_t)t * kTileRows), &ss.full[stage]);
           }
         }
+        filled |= 1u << stage;
+        filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
+      for (int st = 0; st < S; ++st)
+        if (filled & (1u << st)) mbar_drain(&ss.full[st], (filled_parity >> st) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
@@ -284,8 +301,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       for (uint32_t i = t_lo; i < t_hi && !*abort; ++i) {
-        if (!mbar_wait(&ss.tempty[acc], acc_phase ^ 1, abort, status)) break;
-        if (!mbar_wait(&ss.full[stage], phase, abort, status)) break;
+        if (!mbar_wait(&ss.tempty[acc], acc_phase ^ 1, abort, status, a.wait_ns)) break;
+        if (!mbar_wait(&ss.full[stage], phase, abort, status, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
         const uint32_t sb = sa + a_bytes;
@@ -301,6 +318,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (++stage == S) { stage = 0; phase ^= 1; }
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
+      // every MMA this thread issued has completed before the CTA frees TMEM and exits
+      umma_commit(&ss.drain);
+      mbar_drain(&ss.drain, 0);
     }
   } else {
     // ------------------------------ epilogue (warps 2..5) ------------------------------
@@ -341,7 +361,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const int e = t * kTileRows + row;       // position (Full) or slot (Reindex)
       int jpool = -1;                          // Reindex: this slot's pool block
       if (kGather && e < a.pool_blocks * 8) jpool = __ldg(a.pool + (int64_t)q * a.pool_blocks + (e >> 3));
-      bool ok = mbar_wait(&ss.tfull[acc], acc_phase, abort, status);
+      bool ok = mbar_wait(&ss.tfull[acc], acc_phase, abort, status, a.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       float v[32];
       if (ok) {
@@ -673,6 +693,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   __shared__ uint32_t wcnt[kSelThreads / 32];
   __shared__ uint32_t s_base;
   __shared__ int s_last;
+  __shared__ int s_over;
   __shared__ __align__(16) uint32_t hsm[2048];
   __shared__ uint32_t pre[kMaxListChunks + 1];
   __shared__ uint32_t soff[kMaxListChunks];  // list offset of each chunk's candidates
@@ -835,8 +856,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
       uint32_t tot = 0;
       for (int i = 0; i < kSelThreads / 32; ++i) { const uint32_t x = wcnt[i]; wcnt[i] = tot; tot += x; }
       s_base = tot ? atomicAdd(p.fill + r, tot) : 0u;
+      // the histogram bounds the list (n_cand <= cand_cap); keys that disagree with it
+      // (left by an aborted score kernel) must still not write past the list
+      s_over = s_base + tot > (uint32_t)p.cand_cap;
+      if (s_over) report(a.seqs.status, CSA2_ERR_CAPACITY);
       seg[0] = s_base;
-      seg[1] = tot;
+      seg[1] = s_over ? 0u : tot;
     }
     __syncthreads();
     uint32_t o = s_base + wcnt[wid];
@@ -847,7 +872,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
     for (int k = 0; k < kPerLane; ++k) {
       const bool pr = kk[k] != 0u;
       const uint32_t m = __ballot_sync(0xffffffffu, pr);
-      if (pr) {
+      if (pr && !s_over) {
         const uint32_t at = o + __popc(m & lt);
         cand[at] = (uint32_t)(lo + w_lo + 32 * k + lane);
         cand_key[at] = kk[k];
@@ -1060,6 +1085,7 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   sa.block = block;
   sa.hist = reinterpret_cast<uint32_t*>(wsb + L.p[0].hist);
   sa.bhist = brow_len > 0 ? reinterpret_cast<uint32_t*>(wsb + L.p[1].hist) : nullptr;
+  sa.wait_ns = wait_limit_ns();
   const uint32_t stage_bytes = (uint32_t)(d_I / 64) * (kTileRows * 128 + sa.n_pad * 128);
   const int sms = device_sms();
   if (sms <= 0) return CSA2_ERR_CUDA;

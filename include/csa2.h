@@ -313,6 +313,13 @@ CSA2_API const char* csa2_status_string(csa2_status_t status);
 /* The CUDA runtime's message for the latest CUDA failure (a call that returned
  * CSA2_ERR_CUDA) made by the calling host thread, or "no error".  Static storage. */
 CSA2_API const char* csa2_last_cuda_error(void);
+/* Bound, in nanoseconds of the GPU's global timer, of every wait inside the library's
+ * kernels, for launches made after this call (process-wide; 0 restores the default of
+ * 2 s).  A wait that runs out makes its kernel stop every role, wait for the copies and
+ * MMAs it has itself issued, free its tensor memory and record CSA2_ERR_TIMEOUT.  Returns
+ * the previous bound.  Meant for tests of that path and for callers that want a tighter
+ * bound than the default. */
+CSA2_API uint64_t csa2_set_wait_limit_ns(uint64_t ns);
 /* Number of streaming multiprocessors of the current device (0 on error). */
 CSA2_API int32_t csa2_device_sms(void);
 
