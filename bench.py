@@ -247,9 +247,10 @@ def attn_flops(W) -> int:
     return W.num_q * 2 * 2 * W.H * (W.topk + W.window) * W.D
 
 
-def index_bytes(W) -> int:
-    """Indexer-K bytes a Full index call streams: d_I bf16 per visible entry of every query."""
-    return int(np.sum(W.q_visible())) * W.d_I * 2
+def index_bytes(W, esize=2) -> int:
+    """Indexer-K bytes a Full index call streams: d_I elements (bf16: 2 bytes, E4M3: 1) per
+    visible entry of every query."""
+    return int(np.sum(W.q_visible())) * W.d_I * esize
 
 
 def index_flops(W) -> int:
@@ -265,21 +266,25 @@ def attn_launches(W, sms: int) -> int:
 
 
 class Timed:
-    """A workload on the device, its step captured as CUDA graphs (append | Full index | the
-    rest), plus graphs of its index calls alone and of its attention calls alone."""
+    """A workload on the device with its step captured as CUDA graphs: the append, then the
+    whole layer schedule, each layer one csa2_layer_step call (index by its mode, then
+    attention).  Two more graphs hold the Full index call alone and the attention calls
+    alone, for their rooflines."""
 
-    def __init__(self, W, dev, stream):
+    def __init__(self, W, dev, stream, indexer_e4m3=False):
         import torch
         from fp4_kv_cache_03_b200 import csa2, synth
         from fp4_kv_cache_03_b200.workload import DeviceWorkload
         self.W, self.stream = W, stream
-        self.dw = dw = DeviceWorkload(W, device=dev)
+        self.dw = dw = DeviceWorkload(W, device=dev, indexer_e4m3=indexer_e4m3)
         self.full_li = W.modes.index(synth.FULL)
         build_pool = W.pool_blocks > 0
 
         def part_append():
-            if W.append:
-                dw.append(stream=stream)
+            dw.append(stream=stream)
+
+        def part_schedule():                       # (the append has its own graph)
+            dw.run_step(stream=stream, attention=True, via_layer_step=True, append=False)
 
         def part_full():
             L = dw.layers[self.full_li]
@@ -288,23 +293,15 @@ class Timed:
                             pool_blocks=W.pool_blocks if build_pool else 0, block=W.block,
                             pool=dw.pool if build_pool else None, stream=stream)
 
-        def part_rest(attention=True, index=True):
+        def part_attention():
             latest, n_idx = dw.indices[0], 1
             for li, L in enumerate(dw.layers):
                 if L.mode == synth.REINDEX:
-                    idx = dw.indices[n_idx]
+                    latest = dw.indices[n_idx]
                     n_idx += 1
-                    if index:
-                        csa2.index_pool(L.qI, L.w, dw.idx_k, dw.seqs, dw.pool, W.pool_blocks,
-                                        W.block, W.topk, idx, dw.ws_pool, q_visible=dw.q_visible,
-                                        stream=stream)
-                    latest = idx
-                elif L.mode == synth.FULL and li != self.full_li:
-                    raise NotImplementedError("one Full layer per step")
-                if attention:
-                    dw.attend(li, latest, stream=stream)
+                dw.attend(li, latest, stream=stream)
 
-        self.parts = (part_append, part_full, part_rest) if W.append else (part_full, part_rest)
+        self.parts = (part_append, part_schedule) if W.append else (part_schedule,)
         self.graphs = []
         with torch.cuda.stream(stream):
             for fn in self.parts:                      # eager once before capture
@@ -315,10 +312,10 @@ class Timed:
                 with torch.cuda.graph(g, stream=stream):
                     fn()
                 self.graphs.append(g)
-            self.g_attn = torch.cuda.CUDAGraph()       # every attention call of the step
+            self.g_attn = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.g_attn, stream=stream):
-                part_rest(attention=True, index=False)
-            self.g_full = torch.cuda.CUDAGraph()       # the Full index call alone
+                part_attention()
+            self.g_full = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.g_full, stream=stream):
                 part_full()
         stream.synchronize()
@@ -327,28 +324,25 @@ class Timed:
             raise csa2.CSA2Error(st, f"{W.name}: warm-up step")
 
     def release(self):
-        for g in self.graphs + [self.g_attn, self.g_full]:
-            del g
         self.graphs = []
+        self.g_attn = self.g_full = None
+
+    def replay_step(self):
+        for g in self.graphs:
+            g.replay()
 
     def time_steps(self, steps, warmup, flush):
-        """Per-step device times (ms): whole step and its Full index, L2 flushed between."""
+        """Per-step device times (ms), L2 flushed between steps."""
         import torch
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         with torch.cuda.stream(self.stream):
             for k in range(-warmup, steps):
                 flush.zero_()
-                e = evs[k] if k >= 0 else None
-                if e: e[0].record(self.stream)
-                if len(self.graphs) == 3:              # the append
-                    self.graphs[0].replay()
-                if e: e[1].record(self.stream)
-                self.graphs[-2].replay()               # the Full index
-                if e: e[2].record(self.stream)
-                self.graphs[-1].replay()               # the rest of the schedule
-                if e: e[3].record(self.stream)
+                if k >= 0: evs[k][0].record(self.stream)
+                self.replay_step()
+                if k >= 0: evs[k][1].record(self.stream)
         self.stream.synchronize()
-        return [e[0].elapsed_time(e[3]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs]
+        return [a.elapsed_time(b) for a, b in evs]
 
     def time_graph(self, g, reps, flush):
         """Mean device time (s) of one replay of graph g, L2 flushed between replays."""
@@ -364,24 +358,39 @@ class Timed:
         return sum(a.elapsed_time(b) for a, b in ev) / 1e3 / reps
 
 
-def workload_summary(T, steps, warmup, flush, hbm, tflops, sms):
-    """Throughput and rooflines of one workload, from its graphs."""
+def workload_summary(Ts, steps, warmup, flush, hbm, tflops, sms, name=None):
+    """Throughput and rooflines of a workload made of one or more groups (each a Timed),
+    from their graphs; a step runs every group's step in turn."""
+    import torch
     from fp4_kv_cache_03_b200 import csa2, synth
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    stream = Ts[0].stream
+    with torch.cuda.stream(stream):
+        for k in range(-warmup, steps):
+            flush.zero_()
+            if k >= 0: evs[k][0].record(stream)
+            for T in Ts:
+                T.replay_step()
+            if k >= 0: evs[k][1].record(stream)
+    stream.synchronize()
+    t_step = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    units = sum(T.W.num_q * len(T.W.modes) for T in Ts)
+    T = Ts[0]
     W = T.W
     n_layers = len(W.modes)
-    units = W.num_q * n_layers                          # layer-steps per step
-    step_ms, full_ms = T.time_steps(steps, warmup, flush)
-    t_step = statistics.mean(step_ms) / 1e3
-    t_full = statistics.mean(full_ms) / 1e3
+    t_full = T.time_graph(T.g_full, max(3, min(steps, 50)), flush)
     t_attn = T.time_graph(T.g_attn, max(3, min(steps, 50)), flush) / n_layers
-    st = T.dw.status()
-    if st != csa2.OK:
-        raise csa2.CSA2Error(st, f"{W.name}: timed steps")
-    ib, ab = index_bytes(W), attn_alg_bytes(W)
+    for Tg in Ts:
+        st = Tg.dw.status()
+        if st != csa2.OK:
+            raise csa2.CSA2Error(st, f"{Tg.W.name}: timed steps")
+    ib, ab = index_bytes(W, 1 if T.dw.indexer_e4m3 else 2), attn_alg_bytes(W)
     n_index = sum(1 for m in W.modes if m != synth.REUSE)
-    out = {
-        "workload": W.name, "value": units / t_step, "unit": UNIT, "ms_per_step": t_step * 1e3,
-        "layer_steps_per_step": units, "steps": steps,
+    per_group = (1 if W.append else 0) + 3 * n_index + n_layers * attn_launches(W, sms)
+    return {
+        "workload": name or W.name, "value": units / t_step, "unit": UNIT,
+        "ms_per_step": t_step * 1e3, "layer_steps_per_step": units, "steps": steps,
+        "groups": len(Ts), "indexer_k": "e4m3" if T.dw.indexer_e4m3 else "bf16",
         "index_full": {"ms_per_call": t_full * 1e3, "alg_bytes": ib, "achieved_gbs": ib / t_full / 1e9,
                        "frac_hbm": ib / t_full / 1e9 / hbm,
                        "tflops": index_flops(W) / t_full / 1e12},
@@ -389,9 +398,8 @@ def workload_summary(T, steps, warmup, flush, hbm, tflops, sms):
                       "achieved_gbs": ab / t_attn / 1e9, "frac_hbm": ab / t_attn / 1e9 / hbm,
                       "tflops": attn_flops(W) / t_attn / 1e12,
                       "frac_bf16_peak": attn_flops(W) / t_attn / 1e12 / tflops},
-        "gpu_launches_per_step": (1 if W.append else 0) + 3 * n_index + n_layers * attn_launches(W, sms),
+        "gpu_launches_per_step": per_group * len(Ts),
     }
-    return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -413,8 +421,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.zero_()
-            for g in T.graphs:
-                g.replay()
+            T.replay_step()
     stream.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -423,7 +430,7 @@ def run_ours(args, rank, world, local_rank):
     uuid = getattr(props, "uuid", None)
     clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else local_rank)
     clocks.start()
-    step_ms, full_ms = T.time_steps(args.steps, 0, flush)
+    step_ms = T.time_steps(args.steps, 0, flush)
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -453,8 +460,7 @@ def run_ours(args, rank, world, local_rank):
             e2e_ev[k][0].record(stream)
             for h, d in h_in:
                 d.copy_(h, non_blocking=True)
-            for g in T.graphs:
-                g.replay()
+            T.replay_step()
             for h, d in h_out:
                 h.copy_(d, non_blocking=True)
             e2e_ev[k][1].record(stream)
@@ -463,7 +469,7 @@ def run_ours(args, rank, world, local_rank):
 
     # --- the dominant op, sparse attention, and the Full index: their own graphs ---
     t_attn = T.time_graph(T.g_attn, max(3, min(args.steps, 200)), flush) / n_layers
-    t_full = statistics.mean(full_ms) / 1e3
+    t_full = T.time_graph(T.g_full, max(3, min(args.steps, 200)), flush)
     ab = attn_alg_bytes(W)
     attn_achieved = ab / t_attn / 1e9
     ib = index_bytes(W)
@@ -512,13 +518,21 @@ def run_ours(args, rank, world, local_rank):
     # --- the other workloads, same run, same timing rules (fewer steps) ---
     if not args.no_extras and world == 1:
         extras = {}
-        names = [n for n in ("decoder_step_1m", "ragged_decode", "encoder_chunk") if n != W.name]
         k = max(3, min(args.steps, 20))
-        for name in names:
-            T2 = Timed(synth.workload(name), dev, stream)
-            extras[name] = workload_summary(T2, k, 3, flush, hbm, tflops, sms)
-            T2.release()
-            del T2
+        # name: (member workloads, E4M3 indexer K)
+        groups = {"decoder_step_1m": (("decoder_step_1m",), False),
+                  "decoder_step_128k_e4m3_indexer": (("decoder_step_128k",), True),
+                  "decoder_step_1m_e4m3_indexer": (("decoder_step_1m",), True),
+                  "ragged_decode": (("ragged_decode",), False),
+                  "encoder_stack": (synth.ENCODER_STACK, False)}
+        for name, (members, e4m3) in groups.items():
+            if name == W.name:
+                continue
+            Ts = [Timed(synth.workload(m), dev, stream, indexer_e4m3=e4m3) for m in members]
+            extras[name] = workload_summary(Ts, k, 3, flush, hbm, tflops, sms, name=name)
+            for Tg in Ts:
+                Tg.release()
+            del Ts
             torch.cuda.synchronize(dev)
             torch.cuda.empty_cache()
         line["workloads"] = extras

@@ -40,7 +40,7 @@ class Indexer(ctypes.Structure):
     _fields_ = [("qI", c_void_p), ("w", c_void_p), ("H_I", c_int32), ("d_I", c_int32),
                 ("idx_k", c_void_p), ("q_visible", c_void_p), ("max_visible", c_int32),
                 ("pool_blocks", c_int32), ("block", c_int32), ("pool", c_void_p),
-                ("workspace", c_void_p), ("ws_bytes", c_size_t)]
+                ("workspace", c_void_p), ("ws_bytes", c_size_t), ("e4m3", c_int32)]
 
 
 class Attention(ctypes.Structure):
@@ -59,6 +59,16 @@ _SIGS = {
     "csa2_quant_append": (c_int32, [c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
                                     c_int64, c_void_p, c_void_p, c_int32, c_void_p, c_size_t,
                                     c_void_p]),
+    "csa2_quant_append_e4m3k": (c_int32, [c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                          c_int64, c_void_p, c_void_p, c_int32, c_void_p, c_size_t,
+                                          c_void_p]),
+    "csa2_e4m3_from_bf16": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
+    "csa2_index_full_e4m3": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                       c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p,
+                                       c_int32, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa2_index_pool_e4m3": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                       c_int64, Seqs, c_void_p, c_void_p, c_int32, c_int32,
+                                       c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
     "csa2_index_full_workspace": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
     "csa2_index_full": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                   c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p, c_int32,
@@ -165,15 +175,41 @@ def quant_append(x, dst_row, kv_codes, kv_scales, ws, idx_k_in=None, idx_k=None,
                                    ws.numel(), _s(stream)), "csa2_quant_append")
 
 
+def quant_append_e4m3k(x, dst_row, kv_codes, kv_scales, ws, idx_k_in, idx_k, stream=None):
+    """csa2_quant_append with an E4M3 indexer-K cache (``idx_k`` uint8 [cap, d_I])."""
+    assert x.dtype == torch.float32 and dst_row.dtype == torch.int64 and idx_k.dtype == torch.uint8
+    rows, D = x.shape
+    _check(lib().csa2_quant_append_e4m3k(_p(x), rows, D, _p(dst_row), _p(kv_codes), _p(kv_scales),
+                                         kv_codes.shape[0], _u16(idx_k_in), _p(idx_k), idx_k.shape[1],
+                                         _p(ws), ws.numel(), _s(stream)), "csa2_quant_append_e4m3k")
+
+
+def e4m3_from_bf16(x, out=None, stream=None):
+    """bf16 tensor -> E4M3 bytes (uint8, same shape), on the device."""
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    assert out.dtype == torch.uint8 and out.numel() == x.numel()
+    _check(lib().csa2_e4m3_from_bf16(_u16(x), _p(out), x.numel(), _s(stream)), "csa2_e4m3_from_bf16")
+    return out
+
+
 def index_full_workspace(num_q, max_visible, topk, pool_blocks=0, block=8) -> int:
     return int(lib().csa2_index_full_workspace(num_q, max_visible, topk, pool_blocks, block))
 
 
 def index_full(qI, w, idx_k, seqs: Seqs, topk, indices, ws, max_visible, q_visible=None,
                pool_blocks=0, block=8, pool=None, stream=None):
+    """csa2_index_full; with uint8 (E4M3) ``qI`` and ``idx_k``, csa2_index_full_e4m3."""
     num_q, H_I, d_I = qI.shape
     assert w.dtype == torch.float32 and indices.dtype == torch.int32
     assert pool is None or pool.dtype == torch.int32
+    if qI.dtype == torch.uint8:
+        assert idx_k.dtype == torch.uint8
+        _check(lib().csa2_index_full_e4m3(_p(qI), _p(w), num_q, H_I, d_I, _p(idx_k), idx_k.shape[0],
+                                          seqs, _p(q_visible), int(max_visible), topk, _p(indices),
+                                          pool_blocks, block, _p(pool), _p(ws), ws.numel(),
+                                          _s(stream)), "csa2_index_full_e4m3")
+        return
     _check(lib().csa2_index_full(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
                                  seqs, _p(q_visible), int(max_visible), topk, _p(indices),
                                  pool_blocks, block, _p(pool), _p(ws), ws.numel(), _s(stream)),
@@ -208,8 +244,16 @@ def index_pool_workspace(num_q, pool_blocks, block, topk) -> int:
 
 def index_pool(qI, w, idx_k, seqs: Seqs, pool, pool_blocks, block, topk, indices, ws,
                q_visible=None, stream=None):
+    """csa2_index_pool; with uint8 (E4M3) ``qI`` and ``idx_k``, csa2_index_pool_e4m3."""
     num_q, H_I, d_I = qI.shape
     assert w.dtype == torch.float32 and indices.dtype == torch.int32 and pool.dtype == torch.int32
+    if qI.dtype == torch.uint8:
+        assert idx_k.dtype == torch.uint8
+        _check(lib().csa2_index_pool_e4m3(_p(qI), _p(w), num_q, H_I, d_I, _p(idx_k), idx_k.shape[0],
+                                          seqs, _p(q_visible), _p(pool), pool_blocks, block, topk,
+                                          _p(indices), _p(ws), ws.numel(), _s(stream)),
+               "csa2_index_pool_e4m3")
+        return
     _check(lib().csa2_index_pool(_u16(qI), _p(w), num_q, H_I, d_I, _u16(idx_k), idx_k.shape[0],
                                  seqs, _p(q_visible), _p(pool), pool_blocks, block, topk,
                                  _p(indices), _p(ws), ws.numel(), _s(stream)),
@@ -252,10 +296,13 @@ def layer_step(mode, kv_codes, kv_scales, seqs: Seqs, topk, indices, attn: dict,
     ix = None
     if indexer is not None:
         qI = indexer["qI"]
-        ix = Indexer(_u16(qI), _p(indexer["w"]), qI.shape[1], qI.shape[2], _u16(indexer["idx_k"]),
+        e4m3 = qI.dtype == torch.uint8
+        assert e4m3 == (indexer["idx_k"].dtype == torch.uint8)
+        qp, kp = (_p(qI), _p(indexer["idx_k"])) if e4m3 else (_u16(qI), _u16(indexer["idx_k"]))
+        ix = Indexer(qp, _p(indexer["w"]), qI.shape[1], qI.shape[2], kp,
                      _p(indexer.get("q_visible")), int(indexer.get("max_visible", 0)),
                      int(indexer.get("pool_blocks", 0)), int(indexer.get("block", 8)),
-                     _p(indexer.get("pool")), _p(indexer["ws"]), indexer["ws"].numel())
+                     _p(indexer.get("pool")), _p(indexer["ws"]), indexer["ws"].numel(), int(e4m3))
     _check(lib().csa2_layer_step(int(mode), num_q, _p(kv_codes), _p(kv_scales), kv_codes.shape[0],
                                  seqs, topk, _p(indices), ctypes.byref(ix) if ix is not None else None,
                                  ctypes.byref(at), _s(stream)), "csa2_layer_step")

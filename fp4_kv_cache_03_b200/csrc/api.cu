@@ -65,14 +65,27 @@ extern "C" csa2_status_t csa2_layer_step(csa2_mode_t mode, int32_t num_q, const 
     return CSA2_ERR_INVALID_ARG;
   if (!at || (mode != CSA2_MODE_REUSE && !ix)) return CSA2_ERR_INVALID_ARG;
   csa2_status_t st = CSA2_OK;
-  if (mode == CSA2_MODE_FULL) {
-    st = csa2_index_full(ix->qI, ix->w, num_q, ix->H_I, ix->d_I, ix->idx_k, cap_rows, seqs,
-                         ix->q_visible, ix->max_visible, topk, indices, ix->pool_blocks,
-                         ix->block, ix->pool, ix->workspace, ix->ws_bytes, stream);
-  } else if (mode == CSA2_MODE_REINDEX) {
-    st = csa2_index_pool(ix->qI, ix->w, num_q, ix->H_I, ix->d_I, ix->idx_k, cap_rows, seqs,
-                         ix->q_visible, ix->pool, ix->pool_blocks, ix->block, topk, indices,
+  if (mode != CSA2_MODE_REUSE && ix->e4m3 != 0 && ix->e4m3 != 1) return CSA2_ERR_INVALID_ARG;
+  if (mode == CSA2_MODE_FULL && !ix->e4m3) {
+    st = csa2_index_full(static_cast<const uint16_t*>(ix->qI), ix->w, num_q, ix->H_I, ix->d_I,
+                         static_cast<const uint16_t*>(ix->idx_k), cap_rows, seqs, ix->q_visible,
+                         ix->max_visible, topk, indices, ix->pool_blocks, ix->block, ix->pool,
                          ix->workspace, ix->ws_bytes, stream);
+  } else if (mode == CSA2_MODE_FULL) {
+    st = csa2_index_full_e4m3(static_cast<const uint8_t*>(ix->qI), ix->w, num_q, ix->H_I, ix->d_I,
+                              static_cast<const uint8_t*>(ix->idx_k), cap_rows, seqs, ix->q_visible,
+                              ix->max_visible, topk, indices, ix->pool_blocks, ix->block, ix->pool,
+                              ix->workspace, ix->ws_bytes, stream);
+  } else if (mode == CSA2_MODE_REINDEX && !ix->e4m3) {
+    st = csa2_index_pool(static_cast<const uint16_t*>(ix->qI), ix->w, num_q, ix->H_I, ix->d_I,
+                         static_cast<const uint16_t*>(ix->idx_k), cap_rows, seqs, ix->q_visible,
+                         ix->pool, ix->pool_blocks, ix->block, topk, indices, ix->workspace,
+                         ix->ws_bytes, stream);
+  } else if (mode == CSA2_MODE_REINDEX) {
+    st = csa2_index_pool_e4m3(static_cast<const uint8_t*>(ix->qI), ix->w, num_q, ix->H_I, ix->d_I,
+                              static_cast<const uint8_t*>(ix->idx_k), cap_rows, seqs, ix->q_visible,
+                              ix->pool, ix->pool_blocks, ix->block, topk, indices, ix->workspace,
+                              ix->ws_bytes, stream);
   }
   if (st != CSA2_OK) return st;
   return csa2_sparse_attn(at->q, num_q, at->H, at->D, kv_codes, kv_scales, cap_rows, seqs,

@@ -122,7 +122,10 @@ __device__ __forceinline__ int find_row(const uint32_t* rowp, int n, uint32_t i)
   return lo;
 }
 
-template <bool kGather>
+// kESize: bytes per indexer element (2: bf16, 1: E4M3).  Either way an indexer row is moved
+// as 128-byte column chunks (64 bf16 or 128 E4M3 values) in the 128-byte-swizzled layout, and
+// one MMA K-step reads 32 bytes of it (16 bf16 with kind::f16, 32 E4M3 with kind::f8f6f4).
+template <bool kGather, int kESize>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                  const ScoreArgs a) {
@@ -131,7 +134,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* status = a.seqs.status;
 
-  const int halves = a.d_I >> 6;                          // 64-element K chunks
+  const int halves = a.d_I * kESize / 128;                // 128-byte K chunks
+  constexpr int kChunkElems = 128 / kESize;                 // elements per chunk
   const uint32_t a_bytes = (uint32_t)halves * kTileRows * 128;
   const uint32_t b_half = (uint32_t)a.n_pad * 128;
   const uint32_t stage_bytes = a_bytes + (uint32_t)halves * b_half;
@@ -234,9 +238,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                                 (uint32_t)halves * ((uint32_t)a.H_I * 128 + nvalid * 8 * 128));
         __syncwarp();
         for (int h = 0; h < halves; ++h) {
-          if (lane == 0) tma_load_2d(sb + h * b_half, &tm_q, h * 64, q * a.H_I, &ss.full[stage]);
+          if (lane == 0)
+            tma_load_2d(sb + h * b_half, &tm_q, h * kChunkElems, q * a.H_I, &ss.full[stage]);
           if (j >= 0)
-            tma_load_2d(sa + h * (kTileRows * 128) + lane * 1024, &tm_k, h * 64,
+            tma_load_2d(sa + h * (kTileRows * 128) + lane * 1024, &tm_k, h * kChunkElems,
                         (int32_t)(row0 + 8 * (int64_t)j), &ss.full[stage]);
         }
         filled |= 1u << stage;
@@ -276,14 +281,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         mbar_arrive_expect_tx(&ss.full[stage], bytes);
         for (int h = 0; h < halves; ++h) {
-          tma_load_2d(sb + h * b_half, &tm_q, h * 64, q * a.H_I, &ss.full[stage]);
+          tma_load_2d(sb + h * b_half, &tm_q, h * kChunkElems, q * a.H_I, &ss.full[stage]);
           if (kGather) {
             for (int k = 0; k < 16; ++k)
               if (blk_row[k] >= 0)
-                tma_load_2d(sa + h * (kTileRows * 128) + k * 1024, &tm_k, h * 64, blk_row[k],
-                            &ss.full[stage]);
+                tma_load_2d(sa + h * (kTileRows * 128) + k * 1024, &tm_k, h * kChunkElems,
+                            blk_row[k], &ss.full[stage]);
           } else {
-            tma_load_2d(sa + h * (kTileRows * 128), &tm_k, h * 64,
+            tma_load_2d(sa + h * (kTileRows * 128), &tm_k, h * kChunkElems,
                         (int32_t)(row0 + (int64_t)t * kTileRows), &ss.full[stage]);
           }
         }
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0 && t_lo < t_hi) {
-      const uint32_t idesc = idesc_bf16(kTileRows, a.n_pad);
+      const uint32_t idesc = kESize == 2 ? idesc_bf16(kTileRows, a.n_pad) : idesc_e4m3(kTileRows, a.n_pad);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       for (uint32_t i = t_lo; i < t_hi && !*abort; ++i) {
@@ -307,11 +312,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
         const uint32_t sb = sa + a_bytes;
         const uint32_t d = tmem + (uint32_t)(acc * a.n_pad);
-        for (int k = 0; k < (a.d_I >> 4); ++k) {
+        for (int k = 0; k < 4 * halves; ++k) {              // 32-byte K-steps
           const int h = k >> 2, sub = k & 3;
           const uint64_t ad = sdesc_sw128(sa + h * (kTileRows * 128) + sub * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(sb + h * b_half + sub * 32, 16, 1024);
-          umma_bf16(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+          if constexpr (kESize == 2) umma_bf16(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+          else umma_e4m3(d, ad, bd, idesc, k > 0 ? 1u : 0u);
         }
         umma_commit(&ss.empty[stage]);
         umma_commit(&ss.tfull[acc]);
@@ -964,16 +970,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 map over a row-major [rows][cols] array, box = 64 columns x box_rows rows,
-// 128-byte swizzle, out-of-bounds reads as zero.
-bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int box_rows) {
+// 2D map over a row-major [rows][cols] array of bf16 (esize 2) or bytes (esize 1), box =
+// one 128-byte column chunk x box_rows rows, 128-byte swizzle, out-of-bounds reads as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int box_rows, int esize) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+  return fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+            const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1041,10 +1048,11 @@ WsLayout layout_of(int num_q, int64_t row_len, int64_t brow_len, int topk, int p
 
 bool pow2_le32(int b) { return b >= 1 && b <= 32 && (b & (b - 1)) == 0; }
 
-// shared driver for Full (kGather = false) and Reindex (kGather = true)
-template <bool kGather>
-csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, int d_I,
-                        const uint16_t* idx_k, int64_t cap_rows, csa2_seqs_t seqs,
+// shared driver for Full (kGather = false) and Reindex (kGather = true), bf16 (kESize = 2)
+// or E4M3 (kESize = 1) indexer inputs
+template <bool kGather, int kESize = 2>
+csa2_status_t run_index(const void* qI, const float* w, int num_q, int H_I, int d_I,
+                        const void* idx_k, int64_t cap_rows, csa2_seqs_t seqs,
                         const int32_t* q_visible, int max_visible, int topk, int32_t* indices,
                         int pool_blocks, int block, int32_t* pool_out, const int32_t* pool_in,
                         void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -1068,8 +1076,8 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   // ---- scores (+ first-digit histograms) ----
   CUtensorMap tm_k, tm_q;
   const int box_rows = kGather ? 8 : kTileRows;
-  if (!make_map(&tm_k, idx_k, cap_rows, d_I, box_rows)) return CSA2_ERR_CUDA;
-  if (!make_map(&tm_q, qI, (int64_t)num_q * H_I, d_I, H_I)) return CSA2_ERR_CUDA;
+  if (!make_map(&tm_k, idx_k, cap_rows, d_I, box_rows, kESize)) return CSA2_ERR_CUDA;
+  if (!make_map(&tm_q, qI, (int64_t)num_q * H_I, d_I, H_I, kESize)) return CSA2_ERR_CUDA;
   ScoreArgs sa{};
   sa.seqs = sq;
   sa.w = w;
@@ -1086,10 +1094,10 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
   sa.hist = reinterpret_cast<uint32_t*>(wsb + L.p[0].hist);
   sa.bhist = brow_len > 0 ? reinterpret_cast<uint32_t*>(wsb + L.p[1].hist) : nullptr;
   sa.wait_ns = wait_limit_ns();
-  const uint32_t stage_bytes = (uint32_t)(d_I / 64) * (kTileRows * 128 + sa.n_pad * 128);
+  const uint32_t stage_bytes = (uint32_t)(d_I * kESize / 128) * (kTileRows * 128 + sa.n_pad * 128);
   const int sms = device_sms();
   if (sms <= 0) return CSA2_ERR_CUDA;
-  auto kern = score_kernel<kGather>;
+  auto kern = score_kernel<kGather, kESize>;
   for (int q0 = 0; q0 < num_q; q0 += kMaxRowsPerLaunch) {
     sa.q0 = q0;
     sa.num_q = std::min(kMaxRowsPerLaunch, num_q - q0);
@@ -1161,8 +1169,8 @@ csa2_status_t run_index(const uint16_t* qI, const float* w, int num_q, int H_I, 
              : CSA2_ERR_CUDA;
 }
 
-csa2_status_t check_common(const uint16_t* qI, const float* w, int num_q, int H_I, int d_I,
-                           const uint16_t* idx_k, int64_t cap_rows, const csa2_seqs_t& seqs,
+csa2_status_t check_common(const void* qI, const float* w, int num_q, int H_I, int d_I,
+                           const void* idx_k, int64_t cap_rows, const csa2_seqs_t& seqs,
                            int topk, const int32_t* indices) {
   if (num_q < 0 || num_q > 65535 || H_I < 1 || H_I > 32 || (d_I != 64 && d_I != 128))
     return CSA2_ERR_UNSUPPORTED;
@@ -1243,6 +1251,40 @@ extern "C" csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int
   return run_index<true>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, 0x7FFFFFFF,
                          topk, indices, pool_blocks, block, nullptr, pool, workspace, ws_bytes,
                          (cudaStream_t)stream);
+}
+
+extern "C" csa2_status_t csa2_index_full_e4m3(const uint8_t* qI, const float* w, int32_t num_q,
+                                              int32_t H_I, int32_t d_I, const uint8_t* idx_k,
+                                              int64_t cap_rows, csa2_seqs_t seqs,
+                                              const int32_t* q_visible, int32_t max_visible,
+                                              int32_t topk, int32_t* indices, int32_t pool_blocks,
+                                              int32_t block, int32_t* pool, void* workspace,
+                                              size_t ws_bytes, void* stream) {
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices);
+  if (st != CSA2_OK || num_q == 0) return st;
+  if (d_I != 128) return CSA2_ERR_UNSUPPORTED;             // one 128-byte row per entry
+  if ((st = check_ws(workspace)) != CSA2_OK) return st;
+  if ((st = check_full(max_visible, pool_blocks, block, pool)) != CSA2_OK) return st;
+  return run_index<false, 1>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible,
+                             max_visible, topk, indices, pool_blocks, block, pool, nullptr,
+                             workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+extern "C" csa2_status_t csa2_index_pool_e4m3(const uint8_t* qI, const float* w, int32_t num_q,
+                                              int32_t H_I, int32_t d_I, const uint8_t* idx_k,
+                                              int64_t cap_rows, csa2_seqs_t seqs,
+                                              const int32_t* q_visible, const int32_t* pool,
+                                              int32_t pool_blocks, int32_t block, int32_t topk,
+                                              int32_t* indices, void* workspace, size_t ws_bytes,
+                                              void* stream) {
+  csa2_status_t st = check_common(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, topk, indices);
+  if (st != CSA2_OK || num_q == 0) return st;
+  if (d_I != 128) return CSA2_ERR_UNSUPPORTED;
+  if ((st = check_ws(workspace)) != CSA2_OK) return st;
+  if (block != 8 || pool_blocks < 1 || pool_blocks > 8192 || !pool) return CSA2_ERR_UNSUPPORTED;
+  return run_index<true, 1>(qI, w, num_q, H_I, d_I, idx_k, cap_rows, seqs, q_visible, 0x7FFFFFFF,
+                            topk, indices, pool_blocks, block, nullptr, pool, workspace, ws_bytes,
+                            (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------------------------

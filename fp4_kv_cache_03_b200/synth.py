@@ -220,6 +220,13 @@ def workload(name: str) -> Workload:
         return Workload("decoder_step_128k", 1, 1, (131072,), 1, 512, 64, 16, 128, 512, 128,
                         _decoder_modes(5), pool_blocks=2048, block=8, outlier_frac=0.01,
                         append=True)
+    if name.startswith("encoder_group"):
+        # the encoder stack: 3 groups of 6 layers at ratio 2, each group with its own cache
+        # (its Full layer computes its own main KV and indexer K); group g draws its own
+        # streams (seed 3 + 10 g)
+        g = int(name[len("encoder_group"):])
+        return Workload(name, 3 + 10 * g, 1, (32768,), 4096, 512, 64, 16, 128, 512, 128,
+                        (FULL,) + (REUSE,) * 5, ratio=2, q_token0=(61440,))
     if name == "decoder_step_1m":
         return Workload("decoder_step_1m", 2, 1, (1048576,), 1, 512, 64, 16, 128, 512, 128,
                         _decoder_modes(5), pool_blocks=2048, block=8, outlier_frac=0.01,
@@ -229,3 +236,5 @@ def workload(name: str) -> Workload:
 
 WORKLOADS = ("tiny", "decoder_group_128k", "hier_decoder_1m", "encoder_chunk", "ragged_decode",
              "decoder_step_128k", "decoder_step_1m")
+# the 18-layer encoder stack: 3 groups x (Full + 5 Reuse) at ratio 2
+ENCODER_STACK = ("encoder_group0", "encoder_group1", "encoder_group2")

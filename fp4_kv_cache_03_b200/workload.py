@@ -39,7 +39,8 @@ class DeviceWorkload:
 
     STASH_LIMIT = 256 << 20   # keep Reuse stashes for batches whose stash stays this small
 
-    def __init__(self, W: synth.Workload, device="cuda", fill=True, use_stash=True):
+    def __init__(self, W: synth.Workload, device="cuda", fill=True, use_stash=True,
+                 indexer_e4m3=False):
         self.W = W
         self.device = device
         dev = device
@@ -59,6 +60,14 @@ class DeviceWorkload:
         if fill:
             self._fill_cache()
         self.layers = [self._layer_inputs(i, m) for i, m in enumerate(W.modes)]
+        # compact indexer path: E4M3 indexer K (converted from the bf16 cache) and queries
+        self.indexer_e4m3 = indexer_e4m3
+        if indexer_e4m3:
+            self.idx_k = csa2.e4m3_from_bf16(self.idx_k)
+            for L in self.layers:
+                if L.qI is not None:
+                    L.qI = csa2.e4m3_from_bf16(L.qI)
+            torch.cuda.synchronize(dev)
         # outputs / workspaces
         nq = W.num_q
         self.has_pool = W.pool_blocks > 0
@@ -127,13 +136,19 @@ class DeviceWorkload:
 
     # -------------------------------------------------------------------------------
     def append(self, stream=None):
-        csa2.quant_append(self.append_x, self.append_dst, self.kv_codes, self.kv_scales,
-                          self.ws_append, idx_k_in=self.append_k, idx_k=self.idx_k, stream=stream)
+        if self.idx_k.dtype == torch.uint8:
+            csa2.quant_append_e4m3k(self.append_x, self.append_dst, self.kv_codes, self.kv_scales,
+                                    self.ws_append, self.append_k, self.idx_k, stream=stream)
+        else:
+            csa2.quant_append(self.append_x, self.append_dst, self.kv_codes, self.kv_scales,
+                              self.ws_append, idx_k_in=self.append_k, idx_k=self.idx_k, stream=stream)
 
-    def run_step(self, stream=None, attention=True):
-        """One pass of the layer schedule; returns the index tensor each layer used."""
+    def run_step(self, stream=None, attention=True, via_layer_step=False, append=True):
+        """One pass of the layer schedule; returns the index tensor each layer used.
+        With ``via_layer_step`` every layer is one csa2_layer_step call (index + attention
+        by the layer's mode).  ``append=False`` leaves out the step's append."""
         W = self.W
-        if W.append:
+        if W.append and append:
             self.append(stream)
         latest, used, n_idx, pool_built = None, [], 0, False
         for li, L in enumerate(self.layers):
@@ -141,25 +156,51 @@ class DeviceWorkload:
                 idx = self.indices[n_idx]
                 n_idx += 1
                 build = self.has_pool and not pool_built
-                csa2.index_full(L.qI, L.w, self.idx_k, self.seqs, W.topk, idx, self.ws_full,
-                                self.max_visible, q_visible=self.q_visible,
-                                pool_blocks=W.pool_blocks if build else 0, block=W.block,
-                                pool=self.pool if build else None, stream=stream)
+                if via_layer_step and attention:
+                    self.layer_step(li, idx, build_pool=build, stream=stream)
+                else:
+                    csa2.index_full(L.qI, L.w, self.idx_k, self.seqs, W.topk, idx, self.ws_full,
+                                    self.max_visible, q_visible=self.q_visible,
+                                    pool_blocks=W.pool_blocks if build else 0, block=W.block,
+                                    pool=self.pool if build else None, stream=stream)
                 pool_built = pool_built or build
                 latest = idx
             elif L.mode == synth.REINDEX:
                 idx = self.indices[n_idx]
                 n_idx += 1
-                csa2.index_pool(L.qI, L.w, self.idx_k, self.seqs, self.pool, W.pool_blocks,
-                                W.block, W.topk, idx, self.ws_pool, q_visible=self.q_visible,
-                                stream=stream)
+                if via_layer_step and attention:
+                    self.layer_step(li, idx, stream=stream)
+                else:
+                    csa2.index_pool(L.qI, L.w, self.idx_k, self.seqs, self.pool, W.pool_blocks,
+                                    W.block, W.topk, idx, self.ws_pool, q_visible=self.q_visible,
+                                    stream=stream)
                 latest = idx
             else:  # Reuse: no indexer, the latest indices
                 assert latest is not None, "a Reuse layer needs an earlier Full/Reindex layer"
+                if via_layer_step and attention:
+                    self.layer_step(li, latest, stream=stream)
             used.append(latest)
-            if attention:
+            if attention and not via_layer_step:
                 self.attend(li, latest, stream)
         return used
+
+    def layer_step(self, li: int, indices, build_pool=False, stream=None):
+        """Layer li through csa2_layer_step: its mode's indexer (into ``indices``) and
+        attention; a Reuse layer attends with ``indices`` as given."""
+        L, W = self.layers[li], self.W
+        attn = dict(q=L.q, swa_kv=L.swa, swa_start=L.swa_start, q_pos=self.q_pos,
+                    window=W.window, softmax_scale=self.scale, out=self.out[li], lse=self.lse[li],
+                    ws=self.ws_attn, stash=self.stash)
+        ix = None
+        if L.mode == synth.FULL:
+            ix = dict(qI=L.qI, w=L.w, idx_k=self.idx_k, ws=self.ws_full, q_visible=self.q_visible,
+                      max_visible=self.max_visible, pool_blocks=W.pool_blocks if build_pool else 0,
+                      block=W.block, pool=self.pool if build_pool else None)
+        elif L.mode == synth.REINDEX:
+            ix = dict(qI=L.qI, w=L.w, idx_k=self.idx_k, ws=self.ws_pool, q_visible=self.q_visible,
+                      pool_blocks=W.pool_blocks, block=W.block, pool=self.pool)
+        csa2.layer_step(self.MODES[L.mode], self.kv_codes, self.kv_scales, self.seqs, W.topk,
+                        indices, attn, ix, stream=stream)
 
     MODES = {synth.FULL: csa2.MODE_FULL, synth.REINDEX: csa2.MODE_REINDEX, synth.REUSE: csa2.MODE_REUSE}
 

@@ -109,6 +109,16 @@ CSA2_API csa2_status_t csa2_quant_append(const float* x, int32_t rows, int32_t D
                                 uint8_t* kv_codes, uint8_t* kv_scales, int64_t cap_rows,
                                 const uint16_t* idx_k_in, uint16_t* idx_k, int32_t d_I,
                                 void* workspace, size_t ws_bytes, void* stream);
+/* The same append into a compact indexer-K cache: idx_k is E4M3 bytes [cap_rows][d_I]; row r
+ * of the bf16 idx_k_in is converted element by element (round to nearest even, saturating
+ * to +-448; integers in [-16, 16] are exact).  idx_k 8-byte aligned. */
+CSA2_API csa2_status_t csa2_quant_append_e4m3k(const float* x, int32_t rows, int32_t D,
+                                      const int64_t* dst_row, uint8_t* kv_codes, uint8_t* kv_scales,
+                                      int64_t cap_rows, const uint16_t* idx_k_in, uint8_t* idx_k,
+                                      int32_t d_I, void* workspace, size_t ws_bytes, void* stream);
+/* n bf16 values -> n E4M3 bytes (round to nearest even, saturating to +-448): for indexer
+ * queries and bulk indexer-K rows of the compact path. */
+CSA2_API csa2_status_t csa2_e4m3_from_bf16(const uint16_t* in, uint8_t* out, int64_t n, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * a2 + a3 (+ a4).  Full-mode indexer ([MTP] "CSA2：…": Full selects a new Top-512;
@@ -180,6 +190,27 @@ CSA2_API csa2_status_t csa2_index_full_noalloc(const uint16_t* qI, const float* 
 /* Wait for `stream`, then return the status word of the latest csa2_index_full_noalloc call
  * on the current device (CSA2_OK if its kernels recorded no error). */
 CSA2_API csa2_status_t csa2_index_full_noalloc_status(void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Compact indexer K (E4M3): csa2_index_full and csa2_index_pool with qI and idx_k as E4M3
+ * bytes ([num_q][H_I][d_I] and [cap_rows][d_I], d_I = 128, base 16-byte aligned) instead of
+ * bf16.  The score is the same formula over the E4M3 values (fp32 accumulation of the exact
+ * products): for integer-valued indexer inputs in [-16, 16] it, and so every index and pool,
+ * is identical to the bf16 path's, while the Full scan reads 128 instead of 256 bytes per
+ * entry.  The pages put the whole global cache at 890 bytes per token ([OVR] 摘要), which
+ * leaves little room for a 2-byte indexer key.  Workspace sizes are those of the bf16 calls. */
+CSA2_API csa2_status_t csa2_index_full_e4m3(const uint8_t* qI, const float* w, int32_t num_q,
+                                   int32_t H_I, int32_t d_I, const uint8_t* idx_k,
+                                   int64_t cap_rows, csa2_seqs_t seqs, const int32_t* q_visible,
+                                   int32_t max_visible, int32_t topk, int32_t* indices,
+                                   int32_t pool_blocks, int32_t block, int32_t* pool,
+                                   void* workspace, size_t ws_bytes, void* stream);
+CSA2_API csa2_status_t csa2_index_pool_e4m3(const uint8_t* qI, const float* w, int32_t num_q,
+                                   int32_t H_I, int32_t d_I, const uint8_t* idx_k,
+                                   int64_t cap_rows, csa2_seqs_t seqs, const int32_t* q_visible,
+                                   const int32_t* pool, int32_t pool_blocks, int32_t block,
+                                   int32_t topk, int32_t* indices, void* workspace,
+                                   size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * a5. Reindex over the pool ([SURV] §2.2.2: Reindex reuses main KV and indexer K but has
@@ -268,10 +299,10 @@ CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_
  * two structs only group them.  The first error is returned and nothing after it is
  * enqueued.  Only host logic: the work is that of the two calls. */
 typedef struct {
-  const uint16_t* qI;        /* device bf16 [num_q][H_I][d_I] */
+  const void* qI;            /* device [num_q][H_I][d_I]: bf16, or E4M3 bytes when e4m3 */
   const float* w;            /* device fp32 [num_q][H_I] */
   int32_t H_I, d_I;
-  const uint16_t* idx_k;     /* device bf16 [cap_rows][d_I] */
+  const void* idx_k;         /* device [cap_rows][d_I]: bf16, or E4M3 bytes when e4m3 */
   const int32_t* q_visible;  /* device int32 [num_q] or NULL */
   int32_t max_visible;       /* FULL: bound on any query's visible entries */
   int32_t pool_blocks;       /* FULL: 0 = no pool; REINDEX: the pool's blocks per query */
@@ -279,6 +310,7 @@ typedef struct {
   int32_t* pool;             /* FULL: written when pool_blocks > 0; REINDEX: read */
   void* workspace;           /* csa2_index_full_workspace / csa2_index_pool_workspace bytes */
   size_t ws_bytes;
+  int32_t e4m3;              /* 0: bf16 qI / idx_k; 1: the compact E4M3 path */
 } csa2_indexer_t;
 typedef struct {
   const uint16_t* q;         /* device bf16 [num_q][H][D] */

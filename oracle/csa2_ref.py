@@ -167,6 +167,17 @@ def index_scores(qI: np.ndarray, w: np.ndarray, kI: np.ndarray) -> np.ndarray:
     return np.maximum(dots, 0.0) @ np.asarray(w, np.float64)
 
 
+def index_scores_e4m3(qI: np.ndarray, w: np.ndarray, kI: np.ndarray) -> np.ndarray:
+    """The compact indexer (indexer K and Q stored as E4M3 bytes): each value of qI and kI is
+    first rounded to E4M3 (nearest, ties to even, saturating to +-448), then scored exactly
+    as index_scores does.  [OVR] 摘要 puts the whole global cache at 890 bytes per token, which
+    leaves little room for a 2-byte indexer key."""
+    dec = e4m3_decode_table()
+    q8 = dec[e4m3_encode(np.asarray(qI, np.float32))]
+    k8 = dec[e4m3_encode(np.asarray(kI, np.float32))]
+    return index_scores(q8, w, k8)
+
+
 # ============================================================================
 # a3  Top-K selection   [MTP] "CSA2：…" (Full selects a new Top-512)
 # ============================================================================

@@ -12,11 +12,11 @@ from tests import oracle_harness as OH
 pytestmark = pytest.mark.gpu
 
 
-def check(W, queries):
+def check(W, queries, via_layer_step=False):
     from fp4_kv_cache_03_b200 import csa2
     from fp4_kv_cache_03_b200.workload import DeviceWorkload
     dw = DeviceWorkload(W)
-    used = dw.run_step(attention=True)
+    used = dw.run_step(attention=True, via_layer_step=via_layer_step)
     torch.cuda.synchronize()
     assert dw.status() == csa2.OK
     idx = [u.cpu().numpy() for u in used]
@@ -57,5 +57,14 @@ def test_ragged_decode_sampled():
 
 
 def test_decoder_step_128k_sampled():
-    """The 20-layer decoder schedule (Full + pool, 3 Reuse, then 4 x (Reindex + 3 Reuse))."""
-    check(synth.workload("decoder_step_128k"), [0])
+    """The 20-layer decoder schedule (Full + pool, 3 Reuse, then 4 x (Reindex + 3 Reuse)),
+    every layer one csa2_layer_step call."""
+    check(synth.workload("decoder_step_128k"), [0], via_layer_step=True)
+
+
+def test_encoder_stack_via_layer_step():
+    """The 18-layer encoder stack: 3 groups (each its own 32,768-entry cache at ratio 2) of
+    Full + 5 Reuse over a 4,096-query causal chunk, every layer one csa2_layer_step call;
+    sampled queries of every layer of every group against the oracle."""
+    for name in synth.ENCODER_STACK:
+        check(synth.workload(name), [0, 2047, 4095], via_layer_step=True)

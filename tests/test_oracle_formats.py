@@ -182,3 +182,36 @@ def test_page_figures_consistent(golden):
     assert abs(f["kv_bytes_per_token_v41"] * f["ratio_vs_v1"] - f["kv_bytes_per_token_v1"]) \
         < 0.001 * f["kv_bytes_per_token_v1"]
     assert f["pool_blocks"] * f["pool_block_size"] == f["pool_positions"]
+
+
+# ---------------------------------------------------------------------------------------
+# the compact (E4M3) indexer
+# ---------------------------------------------------------------------------------------
+def test_small_integers_round_trip_through_e4m3():
+    """Integers in [-16, 16] need at most 4 significant bits and lie far inside E4M3's
+    normal range, so an E4M3 indexer key holds them exactly."""
+    from oracle import csa2_ref as R
+    v = np.arange(-16, 17, dtype=np.float32)
+    assert np.array_equal(R.e4m3_decode_table()[R.e4m3_encode(v)], v.astype(np.float64))
+    # 17 has 5 significant bits: the nearest E4M3 values are 16 and 18, a tie -> even code 16
+    assert R.e4m3_decode_table()[R.e4m3_encode(np.float32(17.0))] == 16.0
+
+
+def test_e4m3_scores_equal_bf16_scores_on_integer_inputs():
+    from oracle import csa2_ref as R
+    rng = np.random.default_rng(5)
+    qI = rng.integers(-8, 9, size=(16, 128)).astype(np.float64)
+    kI = rng.integers(-8, 9, size=(500, 128)).astype(np.float64)
+    w = rng.integers(1, 5, size=16).astype(np.float64)
+    assert np.array_equal(R.index_scores_e4m3(qI, w, kI), R.index_scores(qI, w, kI))
+
+
+def test_e4m3_scores_round_inputs_first():
+    """Closed forms: 1.1 rounds to 1.125 (the E4M3 grid near 1 steps by 1/8), 500 saturates to
+    448, and a negative dot product is cut by the ReLU."""
+    from oracle import csa2_ref as R
+    qI = np.array([[1.1], [500.0], [-1.0]])
+    w = np.array([1.0, 0.5, 2.0])
+    kI = np.array([[3.0], [1.0]])
+    got = R.index_scores_e4m3(qI, w, kI)
+    assert np.array_equal(got, np.array([1.125 * 3 + 0.5 * 448 * 3, 1.125 + 0.5 * 448]))
