@@ -402,6 +402,45 @@ def workload_summary(Ts, steps, warmup, flush, hbm, tflops, sms, name=None):
     }
 
 
+def compressor_summary(dev, stream, flush, hbm, tflops, steps):
+    """The encoder's sequence compressor fused with the append (csa2_compress_append) at the
+    encoder chunk's size: 65,536 tokens of 512 at ratio 2 -> 32,768 FP4 entries of 512."""
+    import torch
+    from fp4_kv_cache_03_b200 import csa2, synth
+    n, m, D_in, D = 32768, 2, 512, 512
+    bf = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)
+    x = bf(synth.compressor_tokens(11, n * m, D_in))
+    w_t = bf(synth.compressor_map(11, D, m * D_in))
+    dst = torch.arange(n, dtype=torch.int64, device=dev)
+    codes = torch.zeros(n, D // 2, dtype=torch.uint8, device=dev)
+    scales = torch.zeros(n, D // 16, dtype=torch.uint8, device=dev)
+    ws = csa2.workspace(csa2.quant_append_workspace(), dev)
+    with torch.cuda.stream(stream):
+        csa2.compress_append(x, m, w_t, dst, codes, scales, ws, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            csa2.compress_append(x, m, w_t, dst, codes, scales, ws, stream=stream)
+    stream.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(-3, steps):
+            flush.zero_()
+            if k >= 0: ev[k][0].record(stream)
+            g.replay()
+            if k >= 0: ev[k][1].record(stream)
+    stream.synchronize()
+    if csa2.status_fetch(ws) != csa2.OK:
+        raise csa2.CSA2Error(csa2.status_fetch(ws), "compress_append")
+    t = sum(a.elapsed_time(b) for a, b in ev) / 1e3 / steps
+    flops = 2.0 * n * m * D_in * D
+    nbytes = n * m * D_in * 2 + D * m * D_in * 2 + n * (D // 2 + D // 16) + n * 8
+    return {"workload": "compress_append (65,536 tokens x 512 -> 32,768 FP4 entries, ratio 2)",
+            "ms_per_call": t * 1e3, "steps": steps, "gpu_launches_per_step": 1,
+            "tflops": flops / t / 1e12, "frac_bf16_peak": flops / t / 1e12 / tflops,
+            "alg_bytes": nbytes, "achieved_gbs": nbytes / t / 1e9, "frac_hbm": nbytes / t / 1e9 / hbm}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from fp4_kv_cache_03_b200 import csa2, synth
@@ -535,6 +574,7 @@ def run_ours(args, rank, world, local_rank):
             del Ts
             torch.cuda.synchronize(dev)
             torch.cuda.empty_cache()
+        extras["compress_append"] = compressor_summary(dev, stream, flush, hbm, tflops, k)
         line["workloads"] = extras
         if "decoder_step_1m" in extras:
             x = extras["decoder_step_1m"]

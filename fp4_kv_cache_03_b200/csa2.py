@@ -63,6 +63,9 @@ _SIGS = {
                                           c_int64, c_void_p, c_void_p, c_int32, c_void_p, c_size_t,
                                           c_void_p]),
     "csa2_e4m3_from_bf16": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
+    "csa2_compress_append": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_int32,
+                                       c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_size_t,
+                                       c_void_p]),
     "csa2_index_full_e4m3": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                        c_int64, Seqs, c_void_p, c_int32, c_int32, c_void_p,
                                        c_int32, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -182,6 +185,18 @@ def quant_append_e4m3k(x, dst_row, kv_codes, kv_scales, ws, idx_k_in, idx_k, str
     _check(lib().csa2_quant_append_e4m3k(_p(x), rows, D, _p(dst_row), _p(kv_codes), _p(kv_scales),
                                          kv_codes.shape[0], _u16(idx_k_in), _p(idx_k), idx_k.shape[1],
                                          _p(ws), ws.numel(), _s(stream)), "csa2_quant_append_e4m3k")
+
+
+def compress_append(x, m, w_t, dst_row, kv_codes, kv_scales, ws, stream=None):
+    """csa2_compress_append: x bf16 [n_entries * m, D_in] token rows, w_t bf16 [D, m * D_in];
+    entry j goes to cache row dst_row[j]."""
+    assert dst_row.dtype == torch.int64
+    rows, D_in = x.shape
+    D = w_t.shape[0]
+    assert rows % m == 0 and w_t.shape[1] == m * D_in
+    _check(lib().csa2_compress_append(_u16(x), rows // m, m, D_in, _u16(w_t), D, _p(dst_row),
+                                      _p(kv_codes), _p(kv_scales), kv_codes.shape[0], _p(ws),
+                                      ws.numel(), _s(stream)), "csa2_compress_append")
 
 
 def e4m3_from_bf16(x, out=None, stream=None):

@@ -5,24 +5,10 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "fp4_quant.cuh"
 
 namespace csa2 {
 namespace {
-
-// E2M1 magnitude code of q >= 0: nearest of {0,.5,1,1.5,2,3,4,6}, exact midpoints to the
-// even code, saturating at 6.  Each comparison is one threshold of the grid.
-__device__ __forceinline__ uint32_t e2m1_magnitude(float q) {
-  return (uint32_t)(q > 0.25f) + (uint32_t)(q >= 0.75f) + (uint32_t)(q > 1.25f) +
-         (uint32_t)(q >= 1.75f) + (uint32_t)(q > 2.5f) + (uint32_t)(q >= 3.5f) +
-         (uint32_t)(q > 5.0f);
-}
-
-// value of a non-negative E4M3 code (bias 7; exponent field 0 is subnormal m * 2^-9)
-__device__ __forceinline__ float e4m3_value(uint32_t b) {
-  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-  if (e == 0) return (float)m * 0.001953125f;
-  return __uint_as_float(((e + 120u) << 23) | (m << 20));
-}
 
 // kE4M3K: the indexer-K row goes to an E4M3 cache (one byte per element, RNE, saturating),
 // else it is copied as bf16.
@@ -52,19 +38,8 @@ __global__ void __launch_bounds__(256) quant_append_kernel(
         const float4 t = __ldg(src + i);
         v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
       }
-      float amax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const __nv_fp8_storage_t sc =
-          __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
-      const float s = e4m3_value((uint32_t)sc & 0x7Fu);
-      uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t sign = __float_as_uint(v[i]) >> 31;
-        const uint32_t mag = (s != 0.0f) ? e2m1_magnitude(__fdiv_rn(fabsf(v[i]), s)) : 0u;
-        packed[i >> 3] |= ((sign << 3) | mag) << (4 * (i & 7));
-      }
+      uint32_t packed[2];
+      const uint32_t sc = quantize16(v, packed);
       uint2* dc = reinterpret_cast<uint2*>(codes + dst * (int64_t)(D >> 1) + g * 8);
       *dc = make_uint2(packed[0], packed[1]);
       scales[dst * (int64_t)gpr + g] = (uint8_t)sc;

@@ -20,7 +20,8 @@ import numpy as np
 ROW_BLOCK = 4096
 
 # independent random streams, one per kind of input
-S_KV, S_IDXK, S_Q, S_QI, S_W, S_SWA, S_APPEND_X, S_APPEND_K, S_LEN, S_OUTLIER = range(10)
+(S_KV, S_IDXK, S_Q, S_QI, S_W, S_SWA, S_APPEND_X, S_APPEND_K, S_LEN, S_OUTLIER, S_COMP_X,
+ S_COMP_W) = range(12)
 
 
 def _rng(seed: int, stream: int, *more: int) -> np.random.Generator:
@@ -121,6 +122,21 @@ def append_rows(seed: int, step: int, count: int, D: int) -> np.ndarray:
 def append_index_k(seed: int, step: int, count: int, d_I: int) -> np.ndarray:
     r = _rng(seed, S_APPEND_K, step, d_I)
     return _int_to_bf16_bits(r.integers(-8, 9, size=(count, d_I)))
+
+
+def compressor_tokens(seed: int, count: int, D_in: int, lo: int = -8, hi: int = 8) -> np.ndarray:
+    """Token rows entering the sequence compressor: integers in [lo, hi] as bf16 bits."""
+    r = _rng(seed, S_COMP_X, D_in)
+    return _int_to_bf16_bits(r.integers(lo, hi + 1, size=(count, D_in)))
+
+
+def compressor_map(seed: int, D: int, K: int, lo: int = -4, hi: int = 4, shift: int = 6) -> np.ndarray:
+    """The compressor's synthetic linear map, transposed ([D][K]): integers in [lo, hi]
+    times 2^-shift, as bf16 bits (exact).  With integer token rows every fp32 accumulation of
+    the map is exact, so the quantised entries can be compared bit for bit."""
+    r = _rng(seed, S_COMP_W, D, K)
+    v = r.integers(lo, hi + 1, size=(D, K)).astype(np.float32) * np.float32(2.0 ** -shift)
+    return f32_to_bf16_bits(v)
 
 
 def ragged_lengths(seed: int, num_seqs: int, lo: int, hi: int) -> np.ndarray:

@@ -121,6 +121,25 @@ CSA2_API csa2_status_t csa2_quant_append_e4m3k(const float* x, int32_t rows, int
 CSA2_API csa2_status_t csa2_e4m3_from_bf16(const uint16_t* in, uint8_t* out, int64_t n, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * Sequence-axis compressor fused with a1 ([SURV] §2.2.1: every m tokens become one
+ * compressed entry; [MTP] "CSA2：…": the encoder groups run at ratio 2).  The pages do not
+ * give the compressor's form; here it is a linear map of the entry's m token rows:
+ *   entry_j[n] = sum_k xcat_j[k] * w_t[n][k],  xcat_j = [x_{jm}; ...; x_{jm+m-1}], K = m*D_in
+ * (bf16 inputs, fp32 tensor-core accumulation), quantised exactly as csa2_quant_append does
+ * (E4M3 scale of amax/6 per 16 channels, E2M1 codes) into cache row dst_row[j].
+ *   x         device bf16 [n_entries * m][D_in] (token rows, consecutive per entry)
+ *   w_t       device bf16 [D][m * D_in]          m * D_in a multiple of 64
+ *   D         128, 256 or 512
+ *   dst_row   device int64 [n_entries]; rows outside [0, cap_rows) are skipped and
+ *             CSA2_ERR_CAPACITY is recorded
+ *   x, w_t 16-byte aligned; workspace >= CSA2_STATUS_BYTES (status word only) */
+CSA2_API csa2_status_t csa2_compress_append(const uint16_t* x, int32_t n_entries, int32_t m,
+                                   int32_t D_in, const uint16_t* w_t, int32_t D,
+                                   const int64_t* dst_row, uint8_t* kv_codes, uint8_t* kv_scales,
+                                   int64_t cap_rows, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* ---------------------------------------------------------------------------------
  * a2 + a3 (+ a4).  Full-mode indexer ([MTP] "CSA2：…": Full selects a new Top-512;
  * [SURV] §2.2.3: the decoder's first Full layer bounds the search of deeper layers).
  * For query q of sequence s with visible entries V = q_visible[q] (seq_len[s] if

@@ -156,6 +156,26 @@ def bytes_per_entry(D: int) -> int:
 
 
 # ============================================================================
+# sequence-axis compressor  [SURV] §2.2.1 三个压缩维度 (sequence dimension: every m tokens
+#     become one entry; the compressor is inherited from V4); [MTP] "CSA2：…" (encoder groups
+#     at ratio 2).  The pages give no formula: here a linear map of the m token rows.
+# ============================================================================
+
+def compress_rows(x_tokens: np.ndarray, m: int, w_t: np.ndarray) -> np.ndarray:
+    """x_tokens [n*m, D_in] -> entries float64 [n, D]: entry j = concat(x_{jm}, ...,
+    x_{jm+m-1}) @ w_t^T, w_t being the map's transpose [D, m*D_in]."""
+    x = np.asarray(x_tokens, np.float64)
+    n = x.shape[0] // m
+    xcat = x[:n * m].reshape(n, m * x.shape[1])
+    return xcat @ np.asarray(w_t, np.float64).T
+
+
+def compress_quantize(x_tokens: np.ndarray, m: int, w_t: np.ndarray):
+    """The compressor followed by a1: the entries rounded to fp32, then quantize_rows."""
+    return quantize_rows(compress_rows(x_tokens, m, w_t).astype(np.float32))
+
+
+# ============================================================================
 # a2  indexer score     [SURV] §2.2.2 modes table, §2.2.3; [MTP] "CSA2：在层的维度上共享缓存"
 #     (the pages name the indexer; the score formula is a stated reading)
 # ============================================================================
