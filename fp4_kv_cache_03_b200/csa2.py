@@ -32,7 +32,8 @@ class CSA2Error(RuntimeError):
 class Seqs(ctypes.Structure):
     """csa2_seqs_t: ragged batch description (device arrays)."""
     _fields_ = [("num_seqs", c_int32), ("q_per_seq", c_int32),
-                ("seq_start", c_void_p), ("seq_len", c_void_p), ("q_seq", c_void_p)]
+                ("seq_start", c_void_p), ("seq_len", c_void_p), ("q_seq", c_void_p),
+                ("block_table", c_void_p), ("max_pages", c_int32)]
 
 
 class Indexer(ctypes.Structure):
@@ -47,7 +48,7 @@ class Attention(ctypes.Structure):
     """csa2_attention_t: a layer's attention inputs and outputs."""
     _fields_ = [("q", c_void_p), ("H", c_int32), ("D", c_int32), ("swa_kv", c_void_p),
                 ("swa_rows", c_int64), ("swa_start", c_void_p), ("q_pos", c_void_p),
-                ("window", c_int32), ("softmax_scale", c_float), ("out", c_void_p),
+                ("window", c_int32), ("swa_ring", c_int32), ("softmax_scale", c_float), ("out", c_void_p),
                 ("lse", c_void_p), ("kv_stash", c_void_p), ("stash_bytes", c_size_t),
                 ("workspace", c_void_p), ("ws_bytes", c_size_t)]
 
@@ -88,11 +89,16 @@ _SIGS = {
     "csa2_sparse_attn_stash_bytes": (c_size_t, [c_int32, c_int32, c_int32]),
     "csa2_sparse_attn": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                    c_int64, Seqs, c_void_p, c_int32, c_void_p, c_int64, c_void_p,
-                                   c_void_p, c_int32, c_float, c_void_p, c_void_p, c_int32,
+                                   c_void_p, c_int32, c_int32, c_float, c_void_p, c_void_p, c_int32,
                                    c_void_p, c_size_t, c_void_p, c_size_t, c_void_p]),
     "csa2_layer_step": (c_int32, [c_int32, c_int32, c_void_p, c_void_p, c_int64, Seqs, c_int32,
                                   c_void_p, ctypes.POINTER(Indexer), ctypes.POINTER(Attention),
                                   c_void_p]),
+    "csa2_cache_rows": (c_int32, [Seqs, c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
+    "csa2_gather_rows": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_int32, c_void_p,
+                                   c_void_p]),
+    "csa2_scatter_rows": (c_int32, [c_void_p, c_int32, c_void_p, c_int32, c_void_p, c_int64,
+                                    c_void_p]),
     "csa2_status_reset": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_fetch": (c_int32, [c_void_p, c_void_p]),
     "csa2_status_string": (ctypes.c_char_p, [c_int32]),
@@ -147,13 +153,17 @@ def _u16(t):
     return _p(t)
 
 
-def make_seqs(seq_start: torch.Tensor, seq_len: torch.Tensor, q_per_seq: int = 1,
-              q_seq: torch.Tensor | None = None) -> Seqs:
-    """csa2_seqs_t; with ``q_seq`` (int32 [num_q]) each query names its own sequence."""
-    assert seq_start.dtype == torch.int64 and seq_len.dtype == torch.int32
+def make_seqs(seq_start: torch.Tensor | None, seq_len: torch.Tensor, q_per_seq: int = 1,
+              q_seq: torch.Tensor | None = None, block_table: torch.Tensor | None = None) -> Seqs:
+    """csa2_seqs_t; with ``q_seq`` (int32 [num_q]) each query names its own sequence; with
+    ``block_table`` (int32 [num_seqs, max_pages]) the cache is paged (128-row pages)."""
+    assert seq_start is None or seq_start.dtype == torch.int64
+    assert seq_len.dtype == torch.int32
     assert q_seq is None or q_seq.dtype == torch.int32
-    s = Seqs(int(seq_start.numel()), int(q_per_seq), _p(seq_start), _p(seq_len), _p(q_seq))
-    s._keep = (seq_start, seq_len, q_seq)  # keep the tensors alive with the struct
+    assert block_table is None or (block_table.dtype == torch.int32 and block_table.dim() == 2)
+    s = Seqs(int(seq_len.numel()), int(q_per_seq), _p(seq_start), _p(seq_len), _p(q_seq),
+             _p(block_table), int(block_table.shape[1]) if block_table is not None else 0)
+    s._keep = (seq_start, seq_len, q_seq, block_table)  # keep the tensors alive with the struct
     return s
 
 
@@ -284,14 +294,15 @@ def sparse_attn_stash_bytes(num_q, D, topk) -> int:
 
 
 def sparse_attn(q, kv_codes, kv_scales, seqs: Seqs, indices, swa_kv, swa_start, q_pos, window,
-                softmax_scale, out, ws, lse=None, mode=MODE_FULL, stash=None, stream=None):
+                softmax_scale, out, ws, lse=None, mode=MODE_FULL, stash=None, stream=None,
+                swa_ring=0):
     num_q, H, D = q.shape
     topk = indices.shape[1] if indices is not None else 0
     assert out.dtype == torch.float32 and q_pos.dtype == torch.int64
     _check(lib().csa2_sparse_attn(_u16(q), num_q, H, D, _p(kv_codes), _p(kv_scales),
                                   kv_codes.shape[0], seqs, _p(indices), topk, _u16(swa_kv),
                                   swa_kv.shape[0] if swa_kv is not None else 0, _p(swa_start),
-                                  _p(q_pos), window, float(softmax_scale), _p(out), _p(lse),
+                                  _p(q_pos), window, int(swa_ring), float(softmax_scale), _p(out), _p(lse),
                                   int(mode), _p(stash), stash.numel() if stash is not None else 0,
                                   _p(ws), ws.numel(), _s(stream)), "csa2_sparse_attn")
 
@@ -304,7 +315,8 @@ def layer_step(mode, kv_codes, kv_scales, seqs: Seqs, topk, indices, attn: dict,
     q = attn["q"]
     num_q, H, D = q.shape
     at = Attention(_u16(q), H, D, _u16(attn["swa_kv"]), attn["swa_kv"].shape[0], _p(attn["swa_start"]),
-                   _p(attn["q_pos"]), int(attn["window"]), float(attn["softmax_scale"]),
+                   _p(attn["q_pos"]), int(attn["window"]), int(attn.get("swa_ring", 0)),
+                   float(attn["softmax_scale"]),
                    _p(attn["out"]), _p(attn.get("lse")), _p(attn.get("stash")),
                    attn["stash"].numel() if attn.get("stash") is not None else 0,
                    _p(attn["ws"]), attn["ws"].numel())
@@ -321,6 +333,33 @@ def layer_step(mode, kv_codes, kv_scales, seqs: Seqs, topk, indices, attn: dict,
     _check(lib().csa2_layer_step(int(mode), num_q, _p(kv_codes), _p(kv_scales), kv_codes.shape[0],
                                  seqs, topk, _p(indices), ctypes.byref(ix) if ix is not None else None,
                                  ctypes.byref(at), _s(stream)), "csa2_layer_step")
+
+
+def cache_rows(seqs: Seqs, seq, pos, rows=None, stream=None):
+    """Cache rows (int64) of (seq[i], pos[i]) under the layout of ``seqs``; -1 if missing."""
+    assert seq.dtype == torch.int32 and pos.dtype == torch.int32 and seq.numel() == pos.numel()
+    if rows is None:
+        rows = torch.empty(seq.numel(), dtype=torch.int64, device=seq.device)
+    _check(lib().csa2_cache_rows(seqs, _p(seq), _p(pos), seq.numel(), _p(rows), _s(stream)),
+           "csa2_cache_rows")
+    return rows
+
+
+def gather_rows(table, rows, dst=None, stream=None):
+    """dst[i] = table[rows[i]] (a zero row for rows outside the table)."""
+    row_bytes = table.shape[1] * table.element_size()
+    if dst is None:
+        dst = torch.empty((rows.numel(),) + tuple(table.shape[1:]), dtype=table.dtype, device=table.device)
+    _check(lib().csa2_gather_rows(_p(table), table.shape[0], row_bytes, _p(rows), rows.numel(),
+                                  _p(dst), _s(stream)), "csa2_gather_rows")
+    return dst
+
+
+def scatter_rows(src, rows, table, stream=None):
+    """table[rows[i]] = src[i] (rows outside the table are skipped)."""
+    row_bytes = table.shape[1] * table.element_size()
+    _check(lib().csa2_scatter_rows(_p(src), row_bytes, _p(rows), rows.numel(), _p(table),
+                                   table.shape[0], _s(stream)), "csa2_scatter_rows")
 
 
 def status_reset(ws, stream=None) -> None:

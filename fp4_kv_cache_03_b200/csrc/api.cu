@@ -90,6 +90,6 @@ extern "C" csa2_status_t csa2_layer_step(csa2_mode_t mode, int32_t num_q, const 
   if (st != CSA2_OK) return st;
   return csa2_sparse_attn(at->q, num_q, at->H, at->D, kv_codes, kv_scales, cap_rows, seqs,
                           indices, topk, at->swa_kv, at->swa_rows, at->swa_start, at->q_pos,
-                          at->window, at->softmax_scale, at->out, at->lse, mode, at->kv_stash,
+                          at->window, at->swa_ring, at->softmax_scale, at->out, at->lse, mode, at->kv_stash,
                           at->stash_bytes, at->workspace, at->ws_bytes, stream);
 }

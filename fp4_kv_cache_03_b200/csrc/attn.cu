@@ -58,6 +58,8 @@ struct AttnArgs {
   const int32_t* q_seq;                      // or null: q / q_per_seq
   int q_per_seq;
   int num_seqs;
+  const int32_t* block_table;                // paged cache, or null
+  int max_pages;
   const int32_t* indices;
   int topk;
   const uint16_t* swa;
@@ -65,6 +67,7 @@ struct AttnArgs {
   const int64_t* swa_start;
   const int64_t* q_pos;
   int window;
+  int swa_ring;                              // 0: window rows linear; else a ring of this many
   int mode;                                  // csa2_mode_t
   uint8_t* stash;                            // [num_q][n_idx_tiles][stash tile] or null
   int n_idx_tiles;                           // ceil(topk / 128)
@@ -282,8 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // the query's sequence and window: read after the dependency wait, below, once the first
   // tile's index (or stash) loads are in flight
-  int64_t row0 = 0, wrow0 = 0;
-  int slen = 0, n_win = 0;
+  int64_t wrow0 = 0;                         // linear: row of the first window position
+  int64_t wbase = 0;                         // ring: row of ring slot 0
+  int seqv = 0, slen = 0, n_win = 0;
+  int64_t t_q = 0;
 
   // ---- dequantising threads: the FP4 slots this thread loads and converts ----
   // Warp w covers rows 16w .. 16w+15 of an index tile, as two groups of 8 rows: lane l takes
@@ -345,8 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = t * kTile + r;
         const int p = nidx[g];
         vld[g] = false;
+        int64_t grow = -1;
         if (slot < a.topk) {
-          if (p >= 0 && p < slen && row0 + p < a.cap_rows) {
+          if (p >= 0 && p < slen) grow = entry_row(a.seq_start, a.block_table, a.max_pages, seqv, p);
+          if (p >= 0 && p < slen && grow >= 0 && grow < a.cap_rows) {
             vld[g] = true;
           } else if (pl == 0 && (p >= slen || p < -1)) {
             report(a.status, CSA2_ERR_INVALID_ARG);
@@ -355,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (vld[g]) {
-          const uint8_t* crow = a.codes + (row0 + p) * (D / 2) + 16 * pl;
+          const uint8_t* crow = a.codes + grow * (D / 2) + 16 * pl;
 #pragma unroll
           for (int j = 0; j < kSlabs; ++j) cw[g][j] = __ldg(reinterpret_cast<const uint4*>(crow + 64 * j));
-          const uint8_t* srow = a.scales + (row0 + p) * (D / 16);
+          const uint8_t* srow = a.scales + grow * (D / 16);
           uint32_t wv[2 * kSlabs];
           if constexpr (kSlabs >= 2) {
 #pragma unroll
@@ -397,12 +404,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) report(a.status, CSA2_ERR_INVALID_ARG);
       seq = 0;
     }
-    row0 = seq_ok ? a.seq_start[seq] : 0;
+    seqv = seq;
     slen = seq_ok ? a.seq_len[seq] : 0;
-    const int64_t t_q = a.q_pos[q];
+    t_q = a.q_pos[q];
     const int64_t w0 = t_q - a.window + 1 > 0 ? t_q - a.window + 1 : 0;
     n_win = seq_ok ? (int)(t_q + 1 - w0 > 0 ? t_q + 1 - w0 : 0) : 0;
-    wrow0 = (seq_ok && a.window > 0) ? a.swa_start[seq] + w0 : 0;
+    wbase = (seq_ok && a.window > 0) ? a.swa_start[seq] : 0;
+    wrow0 = wbase + w0;
   }
   if (first_fetch && !from_stash) {
     fetch_rows(t_begin, 0);
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // once the previous tile's O MMA has released it
           const int wt = w_lo + i - a.n_idx_tiles;
           // (rows are below 2^31; a start that far outside the map loads zeros only)
-          const int64_t y = wrow0 + (int64_t)wt * kTile;
+          const int64_t y = (a.swa_ring ? wbase : wrow0) + (int64_t)wt * kTile;
           const int32_t y0 = (y < -(int64_t)(1 << 30) || y > (int64_t)0x7FFFFF00) ? -(1 << 30) : (int32_t)y;
           tma_phase = (int)n_tma;
           tma_slabs = 0;
@@ -593,10 +601,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key = qd * 32 + lane;            // this thread's key row = TMEM lane
       bool valid;
       if (win) {
-        const int u = (t - a.n_idx_tiles) * kTile + key;            // window slot
-        const int64_t grow = wrow0 + u;
-        valid = u < n_win && grow >= 0 && grow < a.swa_rows;
-        if (u < n_win && !valid && h0 == 0) report(a.status, CSA2_ERR_CAPACITY);
+        const int u = (t - a.n_idx_tiles) * kTile + key;            // window slot / ring slot
+        if (a.swa_ring) {
+          // ring slot u holds the window position t_q - d, d = (t_q - u) mod ring
+          const int64_t d = ((t_q - u) % a.swa_ring + a.swa_ring) % a.swa_ring;
+          const int64_t grow = wbase + u;
+          const bool in_win = d < n_win;
+          valid = in_win && grow >= 0 && grow < a.swa_rows;
+          if (in_win && !valid && h0 == 0) report(a.status, CSA2_ERR_CAPACITY);
+        } else {
+          const int64_t grow = wrow0 + u;
+          valid = u < n_win && grow >= 0 && grow < a.swa_rows;
+          if (u < n_win && !valid && h0 == 0) report(a.status, CSA2_ERR_CAPACITY);
+        }
       } else {
         valid = ss.valid[k & 1][key] != 0;       // written a tile ahead, before a barrier
       }
@@ -937,11 +954,15 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
                                           const int32_t* indices, int32_t topk,
                                           const uint16_t* swa_kv, int64_t swa_rows,
                                           const int64_t* swa_start, const int64_t* q_pos,
-                                          int32_t window, float softmax_scale, float* out,
+                                          int32_t window, int32_t swa_ring,
+                                          float softmax_scale, float* out,
                                           float* lse, csa2_mode_t mode, void* kv_stash,
                                           size_t stash_bytes, void* workspace, size_t ws_bytes,
                                           void* stream) {
   if (num_q < 0 || topk < 0 || topk > 2048 || window < 0 || window > 1024) return CSA2_ERR_INVALID_ARG;
+  if (swa_ring < 0 || (swa_ring > 0 && (swa_ring % kTile != 0 || swa_ring < window || swa_ring > 1024)))
+    return CSA2_ERR_INVALID_ARG;
+  if (seqs.block_table && seqs.max_pages < 1) return CSA2_ERR_INVALID_ARG;
   if (!attn_shape_ok(H, D)) return CSA2_ERR_UNSUPPORTED;
   if (seqs.num_seqs < 1 ||
       (!seqs.q_seq && (seqs.q_per_seq < 1 || (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)))
@@ -954,7 +975,8 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   if (kv_stash && stash_bytes < csa2_sparse_attn_stash_bytes(num_q, D, topk)) return CSA2_ERR_CAPACITY;
   if (num_q == 0) return CSA2_OK;
   if (num_q > 65535) return CSA2_ERR_UNSUPPORTED;       // queries are a grid dimension
-  if (!q || !out || !q_pos || !seqs.seq_start || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
+  if (!q || !out || !q_pos || !seqs.seq_len) return CSA2_ERR_INVALID_ARG;
+  if (topk > 0 && !seqs.seq_start && !seqs.block_table) return CSA2_ERR_INVALID_ARG;
   if (topk > 0 && (!indices || !kv_codes || !kv_scales || cap_rows <= 0)) return CSA2_ERR_INVALID_ARG;
   if (window > 0 && (!swa_kv || !swa_start || swa_rows < 0)) return CSA2_ERR_INVALID_ARG;
   if (swa_rows > 0x7FFFFFFF) return CSA2_ERR_UNSUPPORTED;    // window rows are TMA coordinates
@@ -966,15 +988,17 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   a.num_q = num_q;
   a.codes = kv_codes; a.scales = kv_scales; a.cap_rows = cap_rows;
   a.seq_start = seqs.seq_start; a.seq_len = seqs.seq_len;
+  a.block_table = seqs.block_table; a.max_pages = seqs.max_pages;
   a.q_seq = seqs.q_seq; a.q_per_seq = seqs.q_per_seq > 0 ? seqs.q_per_seq : 1;
   a.num_seqs = seqs.num_seqs;
   a.indices = indices; a.topk = topk;
   a.swa = swa_kv; a.swa_rows = swa_rows; a.swa_start = swa_start; a.q_pos = q_pos;
   a.window = window;
+  a.swa_ring = window > 0 ? swa_ring : 0;
   a.mode = (int)mode;
   a.stash = static_cast<uint8_t*>(kv_stash);
   a.n_idx_tiles = idx_tiles_of(topk);
-  a.n_win_tiles = (swa_rows > 0) ? win_tiles_of(window) : 0;
+  a.n_win_tiles = (swa_rows > 0 && window > 0) ? (a.swa_ring ? a.swa_ring / kTile : win_tiles_of(window)) : 0;
   a.H = H;
   a.scale_log2 = softmax_scale * kLog2e;
   const int n_tiles = a.n_idx_tiles + a.n_win_tiles;

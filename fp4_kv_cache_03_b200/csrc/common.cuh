@@ -482,6 +482,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------------
+// cache rows: the row of position p of sequence `seq`, linear (seq_start[seq] + p) or paged
+// (block_table[seq][p / 128] * 128 + p % 128); -1 for a page < 0
+// ---------------------------------------------------------------------------------
+constexpr int kPageRows = 128;
+__device__ __forceinline__ int64_t entry_row(const int64_t* seq_start, const int32_t* block_table,
+                                             int max_pages, int seq, int64_t p) {
+  if (!block_table) return seq_start[seq] + p;
+  const int32_t page = __ldg(block_table + (int64_t)seq * max_pages + (p >> 7));
+  return page < 0 ? -1 : (int64_t)page * kPageRows + (p & (kPageRows - 1));
+}
+
+// ---------------------------------------------------------------------------------
 // keys: order-preserving map of fp32 to uint32 (0 is kept free as "no candidate")
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t ordered_key(float s) {

@@ -51,6 +51,8 @@ struct Seqs {
   int num_seqs;
   int max_visible;
   int* status;
+  const int32_t* block_table;      // or null: linear rows from seq_start
+  int max_pages;
 };
 
 // the sequence of query q, or -1 for an out-of-range q_seq value
@@ -59,10 +61,11 @@ __device__ __forceinline__ int seq_of(const Seqs& s, int q) {
   return (seq >= 0 && seq < s.num_seqs) ? seq : -1;
 }
 
-// first cache row of query q's sequence (0 for an invalid sequence, which sees nothing)
-__device__ __forceinline__ int64_t row0_of(const Seqs& s, int q) {
+// cache row of position p of query q's sequence; -1 for an invalid sequence or page (the
+// sequence then sees nothing, or the page's entries are skipped)
+__device__ __forceinline__ int64_t row_of_pos(const Seqs& s, int q, int64_t p) {
   const int seq = seq_of(s, q);
-  return seq >= 0 ? s.seq_start[seq] : 0;
+  return seq >= 0 ? entry_row(s.seq_start, s.block_table, s.max_pages, seq, p) : -1;
 }
 
 __device__ __forceinline__ int visible_of(const Seqs& s, int q) {
@@ -228,10 +231,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
-        const int64_t row0 = row0_of(a.seqs, q);
-        const int j = (lane < 16 && t * 16 + lane < a.pool_blocks)
-                          ? __ldg(a.pool + (int64_t)q * a.pool_blocks + t * 16 + lane)
-                          : -1;
+        int j = (lane < 16 && t * 16 + lane < a.pool_blocks)
+                    ? __ldg(a.pool + (int64_t)q * a.pool_blocks + t * 16 + lane)
+                    : -1;
+        const int64_t brow = j >= 0 ? row_of_pos(a.seqs, q, 8 * (int64_t)j) : -1;
+        if (brow < 0) j = -1;                  // (a block of a missing page loads nothing)
         const uint32_t nvalid = (uint32_t)__popc(__ballot_sync(0xffffffffu, j >= 0));
         if (lane == 0)
           mbar_arrive_expect_tx(&ss.full[stage],
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             tma_load_2d(sb + h * b_half, &tm_q, h * kChunkElems, q * a.H_I, &ss.full[stage]);
           if (j >= 0)
             tma_load_2d(sa + h * (kTileRows * 128) + lane * 1024, &tm_k, h * kChunkElems,
-                        (int32_t)(row0 + 8 * (int64_t)j), &ss.full[stage]);
+                        (int32_t)brow, &ss.full[stage]);
         }
         filled |= 1u << stage;
         filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
@@ -266,17 +270,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (!mbar_wait(&ss.empty[stage], phase ^ 1, abort, status, a.wait_ns)) break;
         uint8_t* sa = base + (size_t)stage * stage_bytes;
         uint8_t* sb = sa + a_bytes;
-        const int64_t row0 = row0_of(a.seqs, q);
         uint32_t bytes = (uint32_t)halves * (uint32_t)a.H_I * 128;
         int32_t blk_row[16];
+        int64_t trow = 0;
         if (kGather) {
           const int32_t* pb = a.pool + (int64_t)q * a.pool_blocks + t * 16;
           for (int k = 0; k < 16; ++k) {
             const int j = (t * 16 + k < a.pool_blocks) ? pb[k] : -1;
-            blk_row[k] = (j >= 0) ? (int32_t)(row0 + 8 * (int64_t)j) : -1;
-            if (j >= 0) bytes += (uint32_t)halves * 8 * 128;
+            const int64_t br = j >= 0 ? row_of_pos(a.seqs, q, 8 * (int64_t)j) : -1;
+            blk_row[k] = (int32_t)br;
+            if (br >= 0) bytes += (uint32_t)halves * 8 * 128;
           }
         } else {
+          // one tile = one page; a missing page loads zeros (outside the map), its keys are
+          // dropped by the epilogue
+          trow = row_of_pos(a.seqs, q, (int64_t)t * kTileRows);
+          if (trow < 0) trow = -(int64_t)(1 << 30);
           bytes += a_bytes;
         }
         mbar_arrive_expect_tx(&ss.full[stage], bytes);
@@ -288,8 +297,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 tma_load_2d(sa + h * (kTileRows * 128) + k * 1024, &tm_k, h * kChunkElems,
                             blk_row[k], &ss.full[stage]);
           } else {
-            tma_load_2d(sa + h * (kTileRows * 128), &tm_k, h * kChunkElems,
-                        (int32_t)(row0 + (int64_t)t * kTileRows), &ss.full[stage]);
+            tma_load_2d(sa + h * (kTileRows * 128), &tm_k, h * kChunkElems, (int32_t)trow,
+                        &ss.full[stage]);
           }
         }
         filled |= 1u << stage;
@@ -367,6 +376,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const int e = t * kTileRows + row;       // position (Full) or slot (Reindex)
       int jpool = -1;                          // Reindex: this slot's pool block
       if (kGather && e < a.pool_blocks * 8) jpool = __ldg(a.pool + (int64_t)q * a.pool_blocks + (e >> 3));
+      // paged cache: entries of a missing page are dropped (and reported)
+      bool page_ok = true;
+      if (a.seqs.block_table) {
+        const int64_t p0 = kGather ? (jpool >= 0 ? 8 * (int64_t)jpool : 0) : (int64_t)t * kTileRows;
+        page_ok = row_of_pos(a.seqs, q, p0) >= 0;
+        if (!page_ok && (kGather ? jpool >= 0 : e < vis)) report(status, CSA2_ERR_CAPACITY);
+      }
       bool ok = mbar_wait(&ss.tfull[acc], acc_phase, abort, status, a.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       float v[32];
@@ -389,15 +405,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       uint32_t key = ordered_key(s);
       if (kGather) {
         if (e < a.pool_blocks * 8) {
-          if (jpool < 0 || 8 * (int64_t)jpool + (e & 7) >= vis) key = 0u;
+          if (jpool < 0 || !page_ok || 8 * (int64_t)jpool + (e & 7) >= vis) key = 0u;
           a.keys[(int64_t)q * a.key_stride + e] = key;
           if (key) atomicAdd(&shist[key >> 21], 1u);
         }
       } else {
-        if (e >= vis) key = 0u;
+        if (e >= vis || !page_ok) key = 0u;
         if (e < vis) {
           a.keys[(int64_t)q * a.key_stride + e] = key;
-          atomicAdd(&shist[key >> 21], 1u);
+          if (key) atomicAdd(&shist[key >> 21], 1u);
         }
         if (a.bkeys) {
           uint32_t m = key;
@@ -1063,7 +1079,8 @@ csa2_status_t run_index(const void* qI, const float* w, int num_q, int H_I, int 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(wsb);
   Seqs sq{seqs.seq_start, seqs.seq_len, q_visible, seqs.q_seq,
-          seqs.q_per_seq > 0 ? seqs.q_per_seq : 1, seqs.num_seqs, max_visible, status};
+          seqs.q_per_seq > 0 ? seqs.q_per_seq : 1, seqs.num_seqs, max_visible, status,
+          seqs.block_table, seqs.max_pages};
 
   {
     const uint32_t n16 = (uint32_t)((L.zero_hi - L.zero_lo) / 16);   // both ends 256-aligned
@@ -1179,8 +1196,9 @@ csa2_status_t check_common(const void* qI, const float* w, int num_q, int H_I, i
   if (seqs.num_seqs < 1 ||
       (!seqs.q_seq && (seqs.q_per_seq < 1 || (int64_t)seqs.num_seqs * seqs.q_per_seq != num_q)))
     return CSA2_ERR_INVALID_ARG;
+  if (seqs.block_table && seqs.max_pages < 1) return CSA2_ERR_INVALID_ARG;
   if (num_q == 0) return CSA2_OK;
-  if (!qI || !w || !idx_k || !indices || !seqs.seq_start || !seqs.seq_len)
+  if (!qI || !w || !idx_k || !indices || (!seqs.seq_start && !seqs.block_table) || !seqs.seq_len)
     return CSA2_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(qI) & 15) || (reinterpret_cast<uintptr_t>(idx_k) & 15))
     return CSA2_ERR_INVALID_ARG;

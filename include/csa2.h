@@ -79,13 +79,23 @@ typedef enum {
  * Query q belongs to sequence q_seq[q] when q_seq is not NULL (any mix of decode queries
  * and chunks of several queries per sequence; a value outside [0, num_seqs) makes that
  * query see nothing and records CSA2_ERR_INVALID_ARG), else to sequence q / q_per_seq, in
- * which case num_seqs * q_per_seq must equal num_q. */
+ * which case num_seqs * q_per_seq must equal num_q.
+ * Cache rows: linear (block_table NULL): position p of sequence s is row seq_start[s] + p.
+ * Paged ([MTP] "FP4 KV 与部署层的几个改动": the global cache outlives the session and is
+ * managed by the serving layer): the cache is a pool of CSA2_PAGE_ROWS-row pages and
+ * position p of sequence s is row block_table[s][p / 128] * 128 + p % 128; seq_start may be
+ * NULL.  Entries of a page < 0 (or beyond the cache) are skipped and CSA2_ERR_CAPACITY is
+ * recorded.  Every index and attention call takes either layout. */
+#define CSA2_PAGE_ROWS 128
 typedef struct {
   int32_t num_seqs;           /* host: number of sequences (>= 1) */
   int32_t q_per_seq;          /* host: queries per sequence when q_seq is NULL (decode: 1) */
-  const int64_t* seq_start;   /* device [num_seqs]: cache row of position 0 */
+  const int64_t* seq_start;   /* device [num_seqs]: cache row of position 0 (linear layout) */
   const int32_t* seq_len;     /* device [num_seqs]: entries stored for the sequence */
   const int32_t* q_seq;       /* device [num_q] or NULL: the sequence of every query */
+  const int32_t* block_table; /* device [num_seqs][max_pages] or NULL: page of positions
+                                 128i .. 128i+127 */
+  int32_t max_pages;          /* host: columns of block_table */
 } csa2_seqs_t;
 
 /* ---------------------------------------------------------------------------------
@@ -257,9 +267,11 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   - for every i with p = indices[q][i] >= 0: the dequantised cache row seq_start[s] + p
  *     (e2m1(code) * e4m3(scale), exact in bf16); p >= seq_len[s] is skipped and
  *     CSA2_ERR_INVALID_ARG recorded;
- *   - the window: swa_kv rows swa_start[s] + u for token positions
- *     u = max(0, t - window + 1) .. t (rows outside [0, swa_rows) are skipped and
- *     CSA2_ERR_CAPACITY recorded).
+ *   - the window: token positions u = max(0, t - window + 1) .. t, at swa_kv row
+ *     swa_start[s] + u (swa_ring = 0), or, with a ring of swa_ring rows per sequence
+ *     (swa_ring a multiple of 128, window <= swa_ring <= 1024), at row
+ *     swa_start[s] + (u mod swa_ring), the ring holding the latest swa_ring tokens (rows
+ *     outside [0, swa_rows) are skipped and CSA2_ERR_CAPACITY recorded).
  * Keys equal values (one vector per row).  Per head h:
  *   l_j = softmax_scale * q[q][h] . row_j;  out[q][h] = sum_j softmax(l)_j row_j;
  *   lse[q][h] = log(sum_j exp(l_j)) (natural log); no rows at all gives out = 0,
@@ -298,7 +310,7 @@ CSA2_API csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int32_
                                const int32_t* indices, int32_t topk,
                                const uint16_t* swa_kv, int64_t swa_rows,
                                const int64_t* swa_start, const int64_t* q_pos,
-                               int32_t window, float softmax_scale,
+                               int32_t window, int32_t swa_ring, float softmax_scale,
                                float* out, float* lse,
                                csa2_mode_t mode, void* kv_stash, size_t stash_bytes,
                                void* workspace, size_t ws_bytes, void* stream);
@@ -339,6 +351,7 @@ typedef struct {
   const int64_t* swa_start;  /* device int64 [num_seqs] */
   const int64_t* q_pos;      /* device int64 [num_q] */
   int32_t window;
+  int32_t swa_ring;          /* 0: linear window rows; else ring rows per sequence */
   float softmax_scale;
   float* out;                /* device fp32 [num_q][H][D] */
   float* lse;                /* device fp32 [num_q][H] or NULL */
@@ -351,6 +364,24 @@ CSA2_API csa2_status_t csa2_layer_step(csa2_mode_t mode, int32_t num_q, const ui
                               const uint8_t* kv_scales, int64_t cap_rows, csa2_seqs_t seqs,
                               int32_t topk, int32_t* indices, const csa2_indexer_t* indexer,
                               const csa2_attention_t* attn, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Paged cache helpers (persistent-cache export and import: [MTP] "FP4 KV 与部署层的几个改动"
+ * -- the global cache is kept for hours, the window is rebuilt, so a sequence's cached
+ * entries move between this cache and slower storage). */
+/* rows[i] = the cache row of position pos[i] of sequence seq[i] under `seqs` (linear or
+ * paged); -1 for a sequence or page that does not exist.  seq, pos device int32 [n]; rows
+ * device int64 [n]. */
+CSA2_API csa2_status_t csa2_cache_rows(csa2_seqs_t seqs, const int32_t* seq, const int32_t* pos,
+                              int32_t n, int64_t* rows, void* stream);
+/* dst[i] = table[rows[i]] for rows of row_bytes bytes (rows[i] outside [0, cap_rows) give a
+ * zero row): e.g. a sequence's FP4 codes, scales or indexer keys into a contiguous buffer
+ * for export.  table, dst 16-byte aligned, row_bytes a multiple of 4. */
+CSA2_API csa2_status_t csa2_gather_rows(const uint8_t* table, int64_t cap_rows, int32_t row_bytes,
+                               const int64_t* rows, int32_t n, uint8_t* dst, void* stream);
+/* table[rows[i]] = src[i] (rows outside [0, cap_rows) are skipped): the import. */
+CSA2_API csa2_status_t csa2_scatter_rows(const uint8_t* src, int32_t row_bytes, const int64_t* rows,
+                                int32_t n, uint8_t* table, int64_t cap_rows, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * Status word helpers. */

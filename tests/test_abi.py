@@ -85,9 +85,9 @@ def test_host_checks_index(L):
 
 def test_host_checks_attention(L):
     from fp4_kv_cache_03_b200 import csa2
-    def call(H=16, D=128, topk=64, window=128, ws=1 << 30, mode=0, stash=None, stash_bytes=0):
+    def call(H=16, D=128, topk=64, window=128, ws=1 << 30, mode=0, stash=None, stash_bytes=0, ring=0):
         return L.csa2_sparse_attn(FAKE, 1, H, D, FAKE, FAKE, 100, _seqs(), FAKE, topk, FAKE, 100,
-                                  FAKE, FAKE, window, 0.1, FAKE, None, mode, stash, stash_bytes,
+                                  FAKE, FAKE, window, ring, 0.1, FAKE, None, mode, stash, stash_bytes,
                                   ctypes.c_void_p(0x100000), ws, None)
     assert call(H=65) == csa2.ERR_UNSUPPORTED
     assert call(H=0) == csa2.ERR_UNSUPPORTED
@@ -96,6 +96,8 @@ def test_host_checks_attention(L):
     assert call(topk=4096) == csa2.ERR_INVALID_ARG
     assert call(ws=300) == csa2.ERR_CAPACITY
     assert call(mode=7) == csa2.ERR_INVALID_ARG
+    assert call(ring=100) == csa2.ERR_INVALID_ARG            # a ring is whole 128-row tiles
+    assert call(ring=128, window=200) == csa2.ERR_INVALID_ARG  # ... at least the window
     assert call(stash=ctypes.c_void_p(0x200000), stash_bytes=16) == csa2.ERR_CAPACITY
     assert call(stash=ctypes.c_void_p(0x200008), stash_bytes=1 << 30) == csa2.ERR_INVALID_ARG
     # 4 tiles of 128 rows: codes (256 B), scales (32 B) and a validity byte per row
@@ -104,7 +106,7 @@ def test_host_checks_attention(L):
     bad = csa2.Seqs(2, 1, FAKE, FAKE)                       # 2 x 1 != 1 query
     mapped = csa2.Seqs(2, 0, FAKE, FAKE, FAKE)             # q_seq given: q_per_seq unused
     args = lambda seqs: (FAKE, 1, 16, 128, FAKE, FAKE, 100, seqs, FAKE, 64, FAKE, 100, FAKE, FAKE,
-                         128, 0.1, FAKE, None, 0, None, 0, ctypes.c_void_p(0x100000), 300, None)
+                         128, 0, 0.1, FAKE, None, 0, None, 0, ctypes.c_void_p(0x100000), 300, None)
     assert L.csa2_sparse_attn(*args(bad)) == csa2.ERR_INVALID_ARG
     assert L.csa2_sparse_attn(*args(mapped)) == csa2.ERR_CAPACITY   # passes the map check
 
@@ -122,7 +124,7 @@ def test_host_checks_layer_step(L):
     import ctypes as C
     from fp4_kv_cache_03_b200 import csa2
     seqs = csa2.Seqs(1, 1, FAKE, FAKE)
-    at = csa2.Attention(FAKE, 16, 128, FAKE, 8, FAKE, FAKE, 4, 0.1, FAKE, None, None, 0, FAKE, 16)
+    at = csa2.Attention(FAKE, 16, 128, FAKE, 8, FAKE, FAKE, 4, 0, 0.1, FAKE, None, None, 0, FAKE, 16)
     ix = csa2.Indexer(FAKE, FAKE, 4, 64, FAKE, None, 4096, 0, 8, None, FAKE, 1 << 30)
 
     def call(mode, ix_, at_, topk=64):
