@@ -32,9 +32,10 @@ namespace {
 
 constexpr int kTileRows = 128;         // entries per MMA tile (M)
 constexpr int kScoreThreads = 192;     // 6 warps
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 512;
 constexpr int kSelChunk = 8192;        // keys per select CTA
 constexpr int kHistBins = 2048;        // first digit: key bits 31..21
+static_assert(kHistBins / 4 == kSelThreads, "one 16-byte piece of a histogram per select thread");
 constexpr int kMaxRowsPerLaunch = 4096;
 constexpr int kMaxListChunks = 1024;   // rows longer than this many chunks stream their keys
 constexpr int kSelSingle = 16384;      // rows up to this long are selected by one CTA
@@ -506,7 +507,7 @@ __device__ void find_bin(const uint32_t* h, int bins, uint32_t k, uint32_t* bin,
                          uint32_t* red) {
   __shared__ uint32_t s_bin, s_above;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int per = bins / kSelThreads;      // contiguous bins per thread (8 or 4)
+  const int per = bins / kSelThreads;      // contiguous bins per thread (4 or 2)
   uint32_t c[8];
   uint32_t mine = 0;
   for (int i = 0; i < per; ++i) { c[i] = h[tid * per + i]; mine += c[i]; }
@@ -686,7 +687,7 @@ __device__ void final_select(const SelProblem& p, int r, const Top& tp, const Sr
     if (!src.pred(key)) continue;
     bool sel = key > T;
     if (!sel && key == T) { sel = taken < my_take; ++taken; }
-    if (sel) {
+    if (sel && o < k) {   // (keys that disagree with the histogram never write past K)
       const uint32_t pos = src.pos_at_ordered(g, c);
       int32_t v = (int32_t)pos;
       if (p.len_mode == 2)
@@ -704,6 +705,170 @@ __global__ void __launch_bounds__(256) ws_zero_kernel(uint4* p, uint32_t n16) {
   pdl_wait();
   for (uint32_t i = blockIdx.x * 256u + threadIdx.x; i < n16; i += gridDim.x * 256u)
     p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// One warp: the bin of the histogram h (32 * kBPL bins) that holds the k-th largest key
+// (1 <= k <= total), the count of keys in the bins above it, and the total (k > total:
+// bin 0, above 0).  Lane l sums the bins [kBPL l, kBPL l + kBPL) with 16-byte loads in
+// rotated order (distinct banks across the warp); a suffix sum over the lanes finds the
+// lane range that holds the k-th key; the warp then splits that range, kBPL / 32 bins per
+// lane, and a second suffix sum finds the bin.  No step walks bins one by one.
+template <int kBPL>
+__device__ __forceinline__ void warp_find_bin(const uint32_t* h, uint32_t k, int lane, uint32_t* bin,
+                                              uint32_t* above, uint32_t* total) {
+  constexpr int kQ = kBPL / 4;               // 16-byte pieces per lane
+  constexpr int kB = kBPL / 32;              // bins per lane in the second step
+  static_assert(kB >= 1 && kQ >= 1, "32 to 64 bins per lane");
+  const uint4* h4 = reinterpret_cast<const uint4*>(h) + lane * kQ;
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) {
+    const uint4 v = h4[(j + lane) & (kQ - 1)];
+    mine += (v.x + v.y) + (v.z + v.w);
+  }
+  uint32_t S = mine;                         // keys in the bins of lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, S, o);
+    if (lane + o < 32) S += y;
+  }
+  *total = __shfl_sync(0xffffffffu, S, 0);
+  const uint32_t who = __ballot_sync(0xffffffffu, S >= k && S - mine < k);
+  if (who == 0u) {
+    *bin = 0u;
+    *above = 0u;
+    return;
+  }
+  const int L = __ffs(who) - 1;
+  const uint32_t runL = __shfl_sync(0xffffffffu, S - mine, L);   // keys above lane L's range
+  uint32_t cb[kB], mb = 0;
+#pragma unroll
+  for (int e = 0; e < kB; ++e) { cb[e] = h[L * kBPL + lane * kB + e]; mb += cb[e]; }
+  uint32_t Sb = mb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, Sb, o);
+    if (lane + o < 32) Sb += y;
+  }
+  const uint32_t kr = k - runL;              // rank of the k-th key inside lane L's range
+  const bool holds = Sb >= kr && Sb - mb < kr;
+  uint32_t b = 0u, ab = 0u;
+  if (holds) {
+    uint32_t run = runL + (Sb - mb);
+#pragma unroll
+    for (int e = kB - 1; e >= 0; --e) {
+      if (run + cb[e] >= k) { b = (uint32_t)(L * kBPL + lane * kB + e); ab = run; break; }
+      run += cb[e];
+    }
+  }
+  const int src = __ffs(__ballot_sync(0xffffffffu, holds)) - 1;
+  *bin = __shfl_sync(0xffffffffu, b, src);
+  *above = __shfl_sync(0xffffffffu, ab, src);
+}
+
+// Block-wide exact Top-K of a row of at most 32 * kSelThreads keys held in shared memory
+// (0 = not a candidate), given the first digit's threshold bin b1 and the count of keys
+// above it.  Thread t owns the contiguous elements [32 t, 32 t + 32); its eight 16-byte
+// pieces are stored swizzled (piece j of run t at 16-byte slot 8 t + (j ^ (t & 7))), so
+// that a warp's loads of piece j hit distinct banks and land in registers with static
+// indices.  One pass marks, as bits, the keys above the threshold bin and in it; the
+// second and third digits (counted in h2 [2048] and h3 [1024], zero on entry), the counts
+// and the ordered write are predicated on those bits, with the keys in registers.  Each
+// digit's bin is found by one warp; one packed scan places the output.  out_of(i) is the
+// output value of element i; n_sel = min(k, valid candidates).
+__device__ __forceinline__ int swz_slot(int t, int j) { return 8 * t + (j ^ (t & 7)); }
+
+template <class OutOf>
+__device__ void resident_select(const uint32_t* keys_s, uint32_t b1, uint32_t above, bool take_all,
+                                uint32_t n_sel, uint32_t k, int32_t* out, uint32_t* h2, uint32_t* h3,
+                                uint32_t* s_res, uint32_t* wcnt, OutOf out_of) {
+  constexpr int kRun = 32;
+  static_assert(kSelThreads * kRun >= kSelSingle, "a run of 32 per thread covers a row");
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  uint32_t kr[kRun];
+#pragma unroll
+  for (int j = 0; j < kRun / 4; ++j) {
+    const uint4 v = reinterpret_cast<const uint4*>(keys_s)[swz_slot(tid, j)];
+    kr[4 * j] = v.x; kr[4 * j + 1] = v.y; kr[4 * j + 2] = v.z; kr[4 * j + 3] = v.w;
+  }
+  // bit i of m_gt / m_eq: element 32 t + i lies above / in the threshold bin (take-all:
+  // every candidate is "above")
+  uint32_t m_gt = 0u, m_eq = 0u;
+#pragma unroll
+  for (int i = 0; i < kRun; ++i) {
+    const uint32_t d = kr[i] >> 21;
+    if (kr[i] != 0u && d > b1) m_gt |= 1u << i;
+    if (kr[i] != 0u && d == b1) m_eq |= 1u << i;
+  }
+  // threshold key T: keys > T are taken, and the first need_eq keys equal to T
+  uint32_t T = 0u, need_eq = 0u;
+  if (take_all) {
+    m_gt |= m_eq;
+    m_eq = 0u;
+  } else {
+    uint32_t krem = n_sel - above;
+    if (m_eq) {
+#pragma unroll
+      for (int i = 0; i < kRun; ++i)
+        if ((m_eq >> i) & 1u) atomicAdd(&h2[(kr[i] >> 10) & 2047u], 1u);
+    }
+    __syncthreads();
+    if (wid == 0) {
+      uint32_t b2, ab, total;
+      warp_find_bin<2048 / 32>(h2, krem, lane, &b2, &ab, &total);
+      if (lane == 0) { s_res[0] = b2; s_res[1] = ab; }
+    }
+    __syncthreads();
+    const uint32_t pre2 = (b1 << 11) | s_res[0];           // key bits 31..10
+    krem -= s_res[1];
+    if (m_eq) {
+#pragma unroll
+      for (int i = 0; i < kRun; ++i)
+        if (((m_eq >> i) & 1u) && (kr[i] >> 10) == pre2) atomicAdd(&h3[kr[i] & 1023u], 1u);
+    }
+    __syncthreads();
+    if (wid == 0) {
+      uint32_t b3, ab, total;
+      warp_find_bin<1024 / 32>(h3, krem, lane, &b3, &ab, &total);
+      if (lane == 0) { s_res[0] = b3; s_res[1] = ab; }
+    }
+    __syncthreads();
+    T = (pre2 << 10) | s_res[0];
+    need_eq = krem - s_res[1];
+  }
+  // one scan of (equal << 16 | greater): the ties taken before this thread are
+  // min(equal rank, need_eq), lowest positions first
+  uint32_t m_tie = 0u;                                     // keys equal to T
+  if (m_eq) {
+#pragma unroll
+    for (int i = 0; i < kRun; ++i) {
+      if (((m_eq >> i) & 1u) && kr[i] > T) m_gt |= 1u << i;
+      if (((m_eq >> i) & 1u) && kr[i] == T) m_tie |= 1u << i;
+    }
+  }
+  const uint32_t my_gt = __popc(m_gt), my_eq = __popc(m_tie);
+  const uint32_t packed = (my_eq << 16) | my_gt;           // block totals < 2^15 each
+  uint32_t incl = packed;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wcnt[wid] = incl;
+  __syncthreads();
+  uint32_t ex = incl - packed;
+  for (int w = 0; w < wid; ++w) ex += wcnt[w];
+  const uint32_t gt_rank = ex & 0xFFFFu, eq_rank = ex >> 16;
+  // the first my_take ties of this run are taken
+  const uint32_t my_take = eq_rank >= need_eq ? 0u : min(my_eq, need_eq - eq_rank);
+  uint32_t m_take = m_tie;
+  for (uint32_t c = my_eq; c > my_take; --c) m_take &= ~(0x80000000u >> __clz(m_take));   // drop the highest
+  uint32_t o = gt_rank + min(eq_rank, need_eq);
+  const uint32_t m_sel = m_gt | m_take;
+  for (uint32_t m = m_sel; m; m &= m - 1u) {
+    if (o >= k) break;                                     // (never past K, even for keys that
+    out[o++] = out_of(tid * kRun + __ffs(m) - 1);          // disagree with the histogram)
+  }
 }
 
 constexpr int kStageCap = 12288;       // candidates staged in shared memory (96 KB)
@@ -726,25 +891,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   if (r >= p.num_rows) return;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   if (p.single) {
-    // Short rows: one CTA holds the row's keys (and, for pool slots, the pool) in shared
-    // memory, compacts the candidates in position order and selects there -- no list in
-    // global memory, no hand-off between CTAs.  The loads go out before the row length is
-    // known; entries at or past it are stale and cleared.
+    // Short rows: one CTA holds the whole row in shared memory and selects there
+    // (resident_select); the first digit's bin comes from the score kernel's histogram,
+    // found by one warp.  Seven block barriers in all.  The loads go out before the row
+    // length is known; entries at or past it are stale and cleared.
     if (c != 0) return;
-    constexpr int kPer = kSelSingle / 4 / kSelThreads;    // 16-byte loads per thread
     uint32_t* keys_s = stage_buf;                          // [kSelSingle]
-    uint32_t* ck = keys_s + kSelSingle;                    // candidates: keys, positions
-    uint32_t* cp = ck + kSelSingle;
-    int32_t* pool_s = reinterpret_cast<int32_t*>(cp + kSelSingle);   // [pool_blocks <= 2048]
-    const uint4* hg = reinterpret_cast<const uint4*>(p.hist + (int64_t)r * kHistBins);
-    const uint4 h0 = hg[tid], h1 = hg[tid + kSelThreads];
+    uint32_t* h2 = keys_s + kSelSingle;                    // [2048] second digit (bits 20..10)
+    uint32_t* h3 = h2 + 2048;                              // [1024] third digit (bits 9..0)
+    int32_t* pool_s = reinterpret_cast<int32_t*>(h3 + 1024);   // [pool_blocks <= 2048]
+    __shared__ uint32_t s_res[3];
+    constexpr int kPer = kSelSingle / 4 / kSelThreads;    // 16-byte loads per thread
+    const uint4 hv = reinterpret_cast<const uint4*>(p.hist + (int64_t)r * kHistBins)[tid];
     const uint4* kg = reinterpret_cast<const uint4*>(p.keys + (int64_t)r * p.stride);
     const int n4 = (int)(p.stride / 4);
     uint4 kv[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int u = tid + j * kSelThreads;
-      kv[j] = u < n4 ? kg[u] : make_uint4(0, 0, 0, 0);
+      kv[j] = u < n4 ? __ldg(kg + u) : make_uint4(0, 0, 0, 0);
     }
     int len;
     if (p.len_mode == 2) {
@@ -761,8 +926,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
       len = row_len(p, a.seqs, r, red);
     }
     len = min(max(len, 0), (int)p.stride);
-    reinterpret_cast<uint4*>(hsm)[tid] = h0;
-    reinterpret_cast<uint4*>(hsm)[tid + kSelThreads] = h1;
+    reinterpret_cast<uint4*>(hsm)[tid] = hv;
+    for (int b = tid; b < 2048 + 1024; b += kSelThreads) h2[b] = 0u;
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int u = tid + j * kSelThreads;
@@ -771,63 +936,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
       if (4 * u + 1 >= len) v.y = 0u;
       if (4 * u + 2 >= len) v.z = 0u;
       if (4 * u + 3 >= len) v.w = 0u;
-      if (u < n4) stage_raw[u] = v;
+      reinterpret_cast<uint4*>(keys_s)[swz_slot(u >> 3, u & 7)] = v;
     }
-    __syncthreads();
-    const Top tp = resolve_top(hsm, (uint32_t)p.k, red);
-    // order-preserving compaction: warp w owns a contiguous run of the row (a multiple of
-    // 256 keys), lane l takes 8 consecutive keys of each 256 (two 16-byte loads) and
-    // counts locally; a warp prefix sum places every lane's candidates in order
-    const int run = ((len + 8 * 256 - 1) / (8 * 256)) * 256;
-    const int w_lo = min(len, wid * run), w_hi = min(len, w_lo + run);
-    auto cand_mask = [&](int i0, uint32_t* kk) -> uint32_t {
-      const int i = i0 + 8 * lane;           // (in the array: i + 7 < kSelSingle; past w_hi masked)
-      const uint4 a0 = i < w_hi ? *reinterpret_cast<const uint4*>(keys_s + i) : make_uint4(0, 0, 0, 0);
-      const uint4 a1 = i + 4 < w_hi ? *reinterpret_cast<const uint4*>(keys_s + i + 4) : make_uint4(0, 0, 0, 0);
-      kk[0] = a0.x; kk[1] = a0.y; kk[2] = a0.z; kk[3] = a0.w;
-      kk[4] = a1.x; kk[5] = a1.y; kk[6] = a1.z; kk[7] = a1.w;
-      uint32_t m = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (i + j < w_hi && kk[j] != 0u && (kk[j] >> 21) >= tp.b1) m |= 1u << j;
-      return m;
-    };
-    uint32_t cnt = 0;
-    for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
-      uint32_t kk[8];
-      cnt += __popc(cand_mask(i0, kk));
+    __syncthreads();                                       // 1
+    const uint32_t k = (uint32_t)p.k;
+    if (wid == 0) {
+      uint32_t b1, ab, total;
+      warp_find_bin<kHistBins / 32>(hsm, k, lane, &b1, &ab, &total);
+      if (lane == 0) { s_res[0] = b1; s_res[1] = ab; s_res[2] = total; }
     }
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) wcnt[wid] = cnt;
-    __syncthreads();
-    uint32_t off = 0, n_cand = 0;
-    for (int w = 0; w < kSelThreads / 32; ++w) {
-      if (w < wid) off += wcnt[w];
-      n_cand += wcnt[w];
-    }
-    for (int i0 = w_lo; i0 < w_hi; i0 += 256) {
-      uint32_t kk[8];
-      const uint32_t m = cand_mask(i0, kk);
-      const uint32_t c = __popc(m);
-      uint32_t incl = c;                     // inclusive prefix over the lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t at = off + incl - c;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (m & (1u << j)) {
-          ck[at] = kk[j];
-          cp[at] = (uint32_t)(i0 + 8 * lane + j);
-          ++at;
-        }
-      off += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    __syncthreads();
-    StagedSource src{ck, cp, n_cand};
-    final_select(p, r, tp, src, red, hsm, p.len_mode == 2 ? pool_s : nullptr);
+    __syncthreads();                                       // 2
+    const uint32_t b1 = s_res[0], n_valid = s_res[2];
+    const bool take_all = n_valid <= k;
+    int32_t* out = p.out + (int64_t)r * p.out_stride;
+    const uint32_t n_sel = min(k, n_valid);
+    for (uint32_t i = n_sel + tid; i < k; i += kSelThreads) out[i] = -1;
+    if (n_sel == 0) return;
+    const int32_t* pmap = p.len_mode == 2 ? pool_s : nullptr;
+    resident_select(keys_s, b1, s_res[1], take_all, n_sel, k, out, h2, h3, s_res, wcnt,
+                    [pmap](int i) -> int32_t { return pmap ? 8 * pmap[i >> 3] + (i & 7) : i; });
     return;
   }
   const int len = row_len(p, a.seqs, r, red);
@@ -838,7 +965,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   // the row's histogram and this chunk's keys, each with one round of independent loads
   {
     const uint4* hg = reinterpret_cast<const uint4*>(p.hist + (int64_t)r * kHistBins);
-    const uint4 h0 = hg[tid], h1 = hg[tid + kSelThreads];
+    const uint4 h0 = hg[tid];                // (one 16-byte piece of the histogram per thread)
     uint4 kv[kSelChunk / 4 / kSelThreads];
     const uint4* kg = reinterpret_cast<const uint4*>(keys + lo);
     const int nv = (hi - lo + 3) / 4;
@@ -848,7 +975,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
       kv[j] = u < nv ? kg[u] : make_uint4(0, 0, 0, 0);
     }
     reinterpret_cast<uint4*>(hsm)[tid] = h0;
-    reinterpret_cast<uint4*>(hsm)[tid + kSelThreads] = h1;
 #pragma unroll
     for (int j = 0; j < kSelChunk / 4 / kSelThreads; ++j) stage_raw[tid + j * kSelThreads] = kv[j];
   }
@@ -857,11 +983,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelArgs a)
   const bool use_list = tp.n_cand <= (uint32_t)p.cand_cap && nch <= kMaxListChunks;
   uint32_t* seg = p.seg + ((int64_t)r * p.chunks + c) * 2;
   if (use_list) {
-    // append this chunk's candidates in position order: warp w owns a contiguous eighth
+    // append this chunk's candidates in position order: warp w owns a contiguous sixteenth
     const int sub = kSelChunk / (kSelThreads / 32);
     const int w_lo = wid * sub, w_hi = min(hi - lo, w_lo + sub);   // chunk-relative
     // this warp's keys in registers (key k of lane l: chunk position w_lo + 32 k + l)
-    constexpr int kPerLane = kSelChunk / kSelThreads;       // 32
+    constexpr int kPerLane = kSelChunk / kSelThreads;       // 16
     uint32_t kk[kPerLane];
 #pragma unroll
     for (int k = 0; k < kPerLane; ++k) {
@@ -1169,17 +1295,12 @@ csa2_status_t run_index(const void* qI, const float* w, int num_q, int H_I, int 
     nprob = 2;
   }
   const dim3 grid(std::max(L.p[0].chunks, nprob == 2 ? L.p[1].chunks : 1), num_q, nprob);
-  // chunked rows: [kStageCap] keys + positions; one-CTA rows: keys, candidate keys and
-  // positions ([kSelSingle] each) and the pool (at most kSelSingle / 8 blocks).  Only a
-  // launch with a one-CTA row asks for the larger size: two chunk CTAs then fit on an SM.
-  bool any_single = sel.p[0].single != 0;
-  if (nprob == 2) any_single = any_single || sel.p[1].single != 0;
-  const size_t sel_smem = any_single ? (size_t)(3 * kSelSingle + kSelSingle / 8) * 4
-                                     : (size_t)2 * kStageCap * 4;
-  // (the function's limit is always the larger size, so that graphs captured with either
-  // launch stay valid)
+  // chunked rows: [kStageCap] keys + positions (96 KB); one-CTA rows: the row's keys, the
+  // second- and third-digit histograms and the pool (at most kSelSingle / 8 blocks): 84 KB
+  static_assert((kSelSingle + 2048 + 1024 + kSelSingle / 8) * 4 <= 2 * kStageCap * 4, "select smem");
+  const size_t sel_smem = (size_t)2 * kStageCap * 4;
   if (checked(cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)((3 * kSelSingle + kSelSingle / 8) * 4))) != cudaSuccess)
+                                   (int)sel_smem)) != cudaSuccess)
     return CSA2_ERR_CUDA;
   return launch_pdl(select_kernel, grid, dim3(kSelThreads), sel_smem, stream, sel) == cudaSuccess
              ? CSA2_OK
