@@ -23,6 +23,7 @@ causal visibility + 6 attention layers), each with the roofline of its index and
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -255,6 +256,25 @@ def index_bytes(W, esize=2) -> int:
 
 def index_flops(W) -> int:
     return int(np.sum(W.q_visible())) * W.H_I * W.d_I * 2
+
+
+def captured_attn_traffic(workload_name: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu capture
+    (profiles/attn_tc_traffic.json), or None when that capture is of another workload or
+    the kernel's sources have changed since it was taken (their SHA-256 differs)."""
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        with open(os.path.join(here, "profiles", "attn_tc_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for rel in rec["source_files"]:
+            with open(os.path.join(here, rel), "rb") as f:
+                h.update(f.read())
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload_name or h.hexdigest() != rec.get("source_sha256"):
+        return None
+    return int(rec["dram_bytes_per_launch"])
 
 
 def attn_launches(W, sms: int) -> int:
@@ -533,8 +553,9 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"kernel": "csa2_sparse_attn (attn_tc_kernel + merge), one layer call",
                      "bound": "hbm", "achieved": attn_achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": attn_achieved / hbm, "traffic": None,
-                     "traffic_note": "DRAM counters are taken in a separate ncu capture (ncu replays kernels)",
+                     "frac": attn_achieved / hbm, "traffic": captured_attn_traffic(W.name),
+                     "traffic_note": "attn_tc_kernel's dram__bytes_read.sum + dram__bytes_write.sum per launch "
+                                     "from the committed ncu capture of these sources (null when they changed)",
                      "peak_source": peak_source,
                      "alg_bytes_per_launch": ab, "alg_bytes_note": "per query: 512 FP4 rows x 288 B + 128 window rows + Q + out, bf16",
                      "fp32_out_extra_bytes": W.num_q * W.H * W.D * 2,
