@@ -7,10 +7,10 @@
 //
 // The key slots of a query form 128-slot tiles: ceil(topk / 128) index tiles (the selected
 // cache rows; slots past topk are empty) and ceil(window / 128) window tiles (its window
-// positions t-W+1 .. t).  One CTA takes a contiguous range of one query's tiles with ALL of
-// its heads (N = 16, 32 or 64 in the MMAs): a tcgen05.mma of M = 128 costs about the same
-// for every N <= 64, so one wide instruction replaces four narrow ones and every selected
-// row is gathered and dequantised once.
+// positions t-W+1 .. t).  One CTA takes a contiguous range of one query's tiles for a group of
+// HN heads (the MMAs' N): 16 when a small batch leaves SMs idle (more CTAs share a query's
+// work), 32, or all 64 from a full wave on.  A tcgen05.mma of M = 128 costs about the same
+// for every N <= 64, and a CTA gathers and dequantises each of its rows once for its heads.
 //
 // Warp roles (288 threads):
 //   warps 0-7  (256 threads) per index tile: thread (row r, half h) prefetches its half of
