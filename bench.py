@@ -285,6 +285,28 @@ def attn_launches(W, sms: int) -> int:
     return 1 + (1 if nsplit > 1 else 0)
 
 
+def coalesce_io(dw):
+    """Lays out the step's per-layer inputs and outputs as slices of a few contiguous device
+    tensors, as a caller that feeds whole steps would hold them: all layers' Q, indexer Q and
+    weights, window rows and outputs each in one tensor.  The end-to-end copies are then one
+    transfer per kind instead of one per layer.  Runs before any graph capture (graphs keep
+    the pointers); returns the tensors by name."""
+    import torch
+    Ls = dw.layers
+    io = {"q": torch.stack([L.q for L in Ls]), "swa": torch.stack([L.swa for L in Ls]),
+          "out": torch.stack(dw.out)}
+    ix = [L for L in Ls if L.qI is not None]
+    if ix:
+        io["qI"] = torch.stack([L.qI for L in ix])
+        io["w"] = torch.stack([L.w for L in ix])
+    for i, L in enumerate(Ls):
+        L.q, L.swa = io["q"][i], io["swa"][i]
+    for j, L in enumerate(ix):
+        L.qI, L.w = io["qI"][j], io["w"][j]
+    dw.out = [io["out"][i] for i in range(len(Ls))]
+    return io
+
+
 class Timed:
     """A workload on the device with its step captured as CUDA graphs: the append, then the
     whole layer schedule, each layer one csa2_layer_step call (index by its mode, then
@@ -297,6 +319,7 @@ class Timed:
         from fp4_kv_cache_03_b200.workload import DeviceWorkload
         self.W, self.stream = W, stream
         self.dw = dw = DeviceWorkload(W, device=dev, indexer_e4m3=indexer_e4m3)
+        self.io = coalesce_io(dw)
         self.full_li = W.modes.index(synth.FULL)
         build_pool = W.pool_blocks > 0
 
@@ -501,15 +524,17 @@ def run_ours(args, rank, world, local_rank):
 
     # --- e2e through the API with host buffers: inputs H2D each step, results D2H ---
     pin = lambda t: t.detach().cpu().pin_memory()
+    # (the step's inputs and outputs are held as a few contiguous tensors: coalesce_io)
+    io = T.io
     h_in = []
     if W.append:
         h_in += [(pin(dw.append_x), dw.append_x), (pin(dw.append_k), dw.append_k)]
-    for L in dw.layers:
-        h_in.append((pin(L.q), L.q))
-        h_in.append((pin(L.swa[-1:]), L.swa[-1:]))      # the step's new window row
-        if L.qI is not None:
-            h_in += [(pin(L.qI), L.qI), (pin(L.w), L.w)]
-    h_out = [(torch.empty_like(o, device="cpu").pin_memory(), o) for o in dw.out]
+    h_in.append((pin(io["q"]), io["q"]))
+    new_rows = io["swa"][:, -1]                        # every layer's new window row
+    h_in.append((pin(new_rows), new_rows))
+    if "qI" in io:
+        h_in += [(pin(io["qI"]), io["qI"]), (pin(io["w"]), io["w"])]
+    h_out = [(torch.empty_like(io["out"], device="cpu").pin_memory(), io["out"])]
     h2d = sum(h.numel() * h.element_size() for h, _ in h_in)
     d2h = sum(h.numel() * h.element_size() for h, _ in h_out)
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
