@@ -44,7 +44,7 @@ namespace {
 constexpr int kDqWarps = 8;                  // dequantise / softmax / epilogue warps
 constexpr int kDqThreads = kDqWarps * 32;
 constexpr int kThreads = kDqThreads + 32;    // + the TMA / MMA warp
-constexpr int kTile = 128;                   // key slots per tile (MMA M of S^T)
+constexpr int kTile = 128;                   // key slots per tile, the larger of the two sizes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;         // rescale O only when a max grows by > 2^8
 
@@ -70,8 +70,8 @@ struct AttnArgs {
   int swa_ring;                              // 0: window rows linear; else a ring of this many
   int mode;                                  // csa2_mode_t
   uint8_t* stash;                            // [num_q][n_idx_tiles][stash tile] or null
-  int n_idx_tiles;                           // ceil(topk / 128)
-  int n_win_tiles;                           // ceil(window / 128)
+  int n_idx_tiles;                           // ceil(topk / kT)
+  int n_win_tiles;                           // ceil(window / kT)
   int H;                                     // real heads
   int hsplit;                                // head groups per query (CTAs of HN heads)
   float scale_log2;                          // softmax_scale * log2(e)
@@ -89,32 +89,31 @@ constexpr uint32_t tmem_cols_for(uint32_t n) {
   return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
 }
 
-// Shared-memory geometry of one CTA (offsets from a 1024-byte aligned base).
-template <int D, int HN>
+// Shared-memory geometry of one CTA (offsets from a 1024-byte aligned base); kT = key
+// slots per tile (64 or 128: the M of the S^T MMA).
+template <int D, int HN, int kT>
 struct Geo {
   static constexpr int kSlabs = D / 128;               // 128-dim slabs (O^T MMA M)
   static constexpr int kChunks = D / 64;               // Q: 64-element (128-byte) chunks
-  static constexpr int kPieces = D / 64;               // 16-byte code pieces per thread
-  static constexpr int kScW = D / 64;                  // 32-bit words of a row's scales
   static constexpr uint32_t kQChunk = HN * 128;        // [HN rows][128 B]
-  // KV tile: D/16 slices of 16 dims, each [128 keys][32 B] with the 32-byte swizzle, so
-  // that one MMA K-step (S^T) or one 16-dim chunk of V^T (O^T) is a contiguous 4 KB
-  static constexpr uint32_t kKVSlice = kTile * 32;
+  // KV tile: D/16 slices of 16 dims, each [kT keys][32 B] with the 32-byte swizzle, so
+  // that one MMA K-step (S^T) or one 16-dim chunk of V^T (O^T) is contiguous
+  static constexpr uint32_t kKVSlice = kT * 32;
   static constexpr uint32_t kKVBytes = (D / 16) * kKVSlice;
   static constexpr uint32_t kPChunk = HN * 128;        // P chunk: [HN heads][64 keys]
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = align1024(kChunks * kQChunk);
   static constexpr uint32_t kOffP = kOffKV + kKVBytes;
-  static constexpr uint32_t kSmem = 1024 + kOffP + 2 * kPChunk;
+  static constexpr uint32_t kSmem = 1024 + kOffP + (kT / 64) * kPChunk;
   static constexpr uint32_t kTmemCols = tmem_cols_for(HN * (1 + kSlabs));   // S^T + O^T
-  // one stash tile: codes [128][D/2], scales [128][D/16], validity [128]
-  static constexpr uint32_t kStashCodes = kTile * (D / 2);
-  static constexpr uint32_t kStashValid = kStashCodes + kTile * (D / 16);
-  static constexpr uint32_t kStashBytes = kStashValid + kTile;
+  // one stash tile: codes [kT][D/2], scales [kT][D/16], validity [kT]
+  static constexpr uint32_t kStashCodes = kT * (D / 2);
+  static constexpr uint32_t kStashValid = kStashCodes + kT * (D / 16);
+  static constexpr uint32_t kStashBytes = kStashValid + kT;
   static_assert(kStashBytes % 16 == 0, "stash tiles stay 16-byte aligned");
 };
 
-template <int HN>
+template <int HN, int kT>
 struct AttnSmem {
   uint64_t bar_q, bar_s, bar_p, bar_o, bar_drain;
   uint64_t full_dq[4], full_tma[4], empty[4];    // per slab
@@ -126,7 +125,7 @@ struct AttnSmem {
   float alpha[HN];
   float red[4][HN];
   int fail;
-  uint8_t valid[2][kTile];                   // slot validity of index tiles k (k even / odd)
+  uint8_t valid[2][kT];                      // slot validity of index tiles k (k even / odd)
 };
 
 // non-negative e4m3 scale byte -> value (bias 7; exponent field 0 is subnormal m * 2^-9)
@@ -221,11 +220,13 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
 // the 256 dequantise / softmax threads only (warp 8 never joins)
 __device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-template <int D, int HN>
+template <int D, int HN, int kT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_swa, const AttnArgs a) {
-  using G = Geo<D, HN>;
+  static_assert(kT == 64 || kT == 128, "64- or 128-key tiles");
+  using G = Geo<D, HN, kT>;
+  constexpr int kG = kT / 64;                // 8-row groups per dequantising warp
   constexpr int kSlabs = G::kSlabs;
   constexpr int HW = HN / 2;                 // heads per warp in softmax and epilogue
   constexpr uint32_t kKVSlice = G::kKVSlice;
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Hr = a.H;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ AttnSmem<HN> ss;
+  __shared__ AttnSmem<HN, kT> ss;
   // 1024-byte aligned base, derived from the shared array itself so that the compiler keeps
   // the shared address space (and knows these buffers do not alias `ss`)
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -291,23 +292,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t t_q = 0;
 
   // ---- dequantising threads: the FP4 slots this thread loads and converts ----
-  // Warp w covers rows 16w .. 16w+15 of an index tile, as two groups of 8 rows: lane l takes
-  // row 16w + 8g + (l & 7) of group g, and of each 128-dim slab j the 16-byte piece
-  // pq = 4j + (l >> 3) (32 dims).  A warp load then reads 8 rows x 64 contiguous bytes, and a
-  // warp store of one 16-byte unit hits 8 rows x 4 slices, which the 32-byte swizzle spreads
-  // over all banks.
+  // Warp w covers rows 8kG w .. 8kG w + 8kG - 1 of an index tile (kG = kT / 64 groups of 8
+  // rows): lane l takes row 8kG w + 8g + (l & 7) of group g, and of each 128-dim slab j the
+  // 16-byte piece pq = 4j + (l >> 3) (32 dims).  A warp load then reads 8 rows x 64
+  // contiguous bytes, and a warp store of one 16-byte unit hits 8 rows x 4 slices, which the
+  // 32-byte swizzle spreads over all banks.
   const int pl = lane >> 3;                  // piece of the slab (0..3)
-  auto row_of = [&](int g) { return 16 * warp + 8 * g + (lane & 7); };
+  auto row_of = [&](int g) { return 8 * kG * warp + 8 * g + (lane & 7); };
   const bool from_stash = a.stash != nullptr && a.mode == CSA2_MODE_REUSE;
   const bool to_stash = a.stash != nullptr && a.mode != CSA2_MODE_REUSE && hg == 0;
-  uint4 cw[2][kSlabs];                       // codes of (row group, slab)
-  uint32_t sc[2][kSlabs];                    // their two scale bytes (low: first 16 dims)
-  bool vld[2] = {false, false};
-  int32_t nidx[2] = {-1, -1};                // indices of the next tile to fetch
+  uint4 cw[kG][kSlabs];                      // codes of (row group, slab)
+  uint32_t sc[kG][kSlabs];                   // their two scale bytes (low: first 16 dims)
+  bool vld[kG];
+  int32_t nidx[kG];                          // indices of the next tile to fetch
+#pragma unroll
+  for (int g = 0; g < kG; ++g) { vld[g] = false; nidx[g] = -1; }
+  // a thread's scale pairs in a stash tile: kSc 16-bit values, (group, slab) in that order
+  constexpr int kSc = kG * kSlabs;
   auto fetch_index = [&](int t) {
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const int slot = t * kTile + row_of(g);
+    for (int g = 0; g < kG; ++g) {
+      const int slot = t * kT + row_of(g);
       nidx[g] = (!from_stash && slot < a.topk) ? __ldg(a.indices + (int64_t)q * a.topk + slot) : -1;
     }
   };
@@ -324,30 +329,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto fetch_rows = [&](int t, int k) {
     if (from_stash) {
       const uint8_t* st = a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStashBytes;
-      const uint4* sp = reinterpret_cast<const uint4*>(st) + (size_t)warp * (2 * kSlabs) * 32 + lane;
+      const uint4* sp = reinterpret_cast<const uint4*>(st) + (size_t)warp * (kG * kSlabs) * 32 + lane;
 #pragma unroll
-      for (int g = 0; g < 2; ++g)
+      for (int g = 0; g < kG; ++g)
 #pragma unroll
         for (int j = 0; j < kSlabs; ++j) cw[g][j] = __ldg(sp + (g * kSlabs + j) * 32);
-      const uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (8 * kSlabs / 2);
-      if constexpr (kSlabs == 4) {
+      const uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (2 * kSc);
+      uint32_t wv[(kSc + 1) / 2];
+      if constexpr (kSc == 8) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(ssc));
-        sc[0][0] = v.x & 0xFFFFu; sc[0][1] = v.x >> 16; sc[0][2] = v.y & 0xFFFFu; sc[0][3] = v.y >> 16;
-        sc[1][0] = v.z & 0xFFFFu; sc[1][1] = v.z >> 16; sc[1][2] = v.w & 0xFFFFu; sc[1][3] = v.w >> 16;
-      } else if constexpr (kSlabs == 2) {
+        wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
+      } else if constexpr (kSc == 4) {
         const uint2 v = __ldg(reinterpret_cast<const uint2*>(ssc));
-        sc[0][0] = v.x & 0xFFFFu; sc[0][1] = v.x >> 16; sc[1][0] = v.y & 0xFFFFu; sc[1][1] = v.y >> 16;
+        wv[0] = v.x; wv[1] = v.y;
+      } else if constexpr (kSc == 2) {
+        wv[0] = __ldg(reinterpret_cast<const uint32_t*>(ssc));
       } else {
-        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(ssc));
-        sc[0][0] = v & 0xFFFFu; sc[1][0] = v >> 16;
+        wv[0] = __ldg(reinterpret_cast<const unsigned short*>(ssc));
       }
 #pragma unroll
-      for (int g = 0; g < 2; ++g) vld[g] = st[G::kStashValid + row_of(g)] != 0;
+      for (int g = 0; g < kG; ++g)
+#pragma unroll
+        for (int j = 0; j < kSlabs; ++j) {
+          const int i = g * kSlabs + j;
+          sc[g][j] = (wv[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+        }
+#pragma unroll
+      for (int g = 0; g < kG; ++g) vld[g] = st[G::kStashValid + row_of(g)] != 0;
     } else {
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
+      for (int g = 0; g < kG; ++g) {
         const int r = row_of(g);
-        const int slot = t * kTile + r;
+        const int slot = t * kT + r;
         const int p = nidx[g];
         vld[g] = false;
         int64_t grow = -1;
@@ -386,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (pl == 0) {
 #pragma unroll
-      for (int g = 0; g < 2; ++g) ss.valid[k & 1][row_of(g)] = vld[g] ? 1 : 0;
+      for (int g = 0; g < kG; ++g) ss.valid[k & 1][row_of(g)] = vld[g] ? 1 : 0;
     }
   };
   // The first index tile's index (or stash rows) goes out first; then the sequence lookups;
@@ -427,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kDqWarps) {
     // =============================== TMA + MMA issue ===============================
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(kTile, HN);                 // KV, Q both K-major
-      const uint32_t idesc_o = idesc_bf16(kTile, HN, true, false);    // V^T MN-major, P K-major
+      const uint32_t idesc_s = idesc_bf16(kT, HN);                    // KV, Q both K-major
+      const uint32_t idesc_o = idesc_bf16(128, HN, true, false);      // V^T (128-dim slab) MN-major, P K-major
       const uint64_t kv_desc = sdesc_sw32(smem_u32(sKV), kKVSlice, 256);
       const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t p_desc = sdesc_sw128(smem_u32(sP), 16, 1024);
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // once the previous tile's O MMA has released it
           const int wt = w_lo + i - a.n_idx_tiles;
           // (rows are below 2^31; a start that far outside the map loads zeros only)
-          const int64_t y = (a.swa_ring ? wbase : wrow0) + (int64_t)wt * kTile;
+          const int64_t y = (a.swa_ring ? wbase : wrow0) + (int64_t)wt * kT;
           const int32_t y0 = (y < -(int64_t)(1 << 30) || y > (int64_t)0x7FFFFF00) ? -(1 << 30) : (int32_t)y;
           tma_phase = (int)n_tma;
           tma_slabs = 0;
@@ -486,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O^T += V^T . P^T, slab by slab; each slab is released when its MMAs complete
         for (int j = 0; j < kSlabs; ++j) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
+          for (int kk = 0; kk < kT / 16; ++kk) {
             const uint32_t poff = (uint32_t)(kk >> 2) * G::kPChunk + (kk & 3) * 32;
             const uint32_t off = (uint32_t)(8 * j) * kKVSlice + kk * 512;   // 16 keys = 2 atoms
             umma_bf16(tO + j * HN, kv_desc + (off >> 4), p_desc + (poff >> 4), idesc_o,
@@ -526,23 +539,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (to_stash && ok) {
           // the stash holds the tile in this thread order, so a Reuse layer's loads coalesce
           uint8_t* st = a.stash + ((int64_t)q * a.n_idx_tiles + t) * G::kStashBytes;
-          uint4* sp = reinterpret_cast<uint4*>(st) + (size_t)warp * (2 * kSlabs) * 32 + lane;
+          uint4* sp = reinterpret_cast<uint4*>(st) + (size_t)warp * (kG * kSlabs) * 32 + lane;
 #pragma unroll
-          for (int g = 0; g < 2; ++g)
+          for (int g = 0; g < kG; ++g)
 #pragma unroll
             for (int j = 0; j < kSlabs; ++j) sp[(g * kSlabs + j) * 32] = cw[g][j];
-          uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (8 * kSlabs / 2);
-          if constexpr (kSlabs == 4) {
-            *reinterpret_cast<uint4*>(ssc) = make_uint4(sc[0][0] | (sc[0][1] << 16), sc[0][2] | (sc[0][3] << 16),
-                                                        sc[1][0] | (sc[1][1] << 16), sc[1][2] | (sc[1][3] << 16));
-          } else if constexpr (kSlabs == 2) {
-            *reinterpret_cast<uint2*>(ssc) = make_uint2(sc[0][0] | (sc[0][1] << 16), sc[1][0] | (sc[1][1] << 16));
+          uint8_t* ssc = st + G::kStashCodes + (size_t)(warp * 32 + lane) * (2 * kSc);
+          uint32_t wv[(kSc + 1) / 2];
+#pragma unroll
+          for (int w = 0; w < (kSc + 1) / 2; ++w) wv[w] = 0u;
+#pragma unroll
+          for (int g = 0; g < kG; ++g)
+#pragma unroll
+            for (int j = 0; j < kSlabs; ++j) {
+              const int i = g * kSlabs + j;
+              wv[i >> 1] |= sc[g][j] << (16 * (i & 1));
+            }
+          if constexpr (kSc == 8) {
+            *reinterpret_cast<uint4*>(ssc) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          } else if constexpr (kSc == 4) {
+            *reinterpret_cast<uint2*>(ssc) = make_uint2(wv[0], wv[1]);
+          } else if constexpr (kSc == 2) {
+            *reinterpret_cast<uint32_t*>(ssc) = wv[0];
           } else {
-            *reinterpret_cast<uint32_t*>(ssc) = sc[0][0] | (sc[1][0] << 16);
+            *reinterpret_cast<unsigned short*>(ssc) = (unsigned short)wv[0];
           }
           if (pl == 0) {
 #pragma unroll
-            for (int g = 0; g < 2; ++g) st[G::kStashValid + row_of(g)] = vld[g] ? 1 : 0;
+            for (int g = 0; g < kG; ++g) st[G::kStashValid + row_of(g)] = vld[g] ? 1 : 0;
           }
         }
         // dequantise slab by slab into the swizzled tile as the previous tile's O MMA
@@ -557,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) {
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
+            for (int g = 0; g < kG; ++g) {
               const uint4 c4 = cw[g][0];
               const float s0 = e4m3_val(sc[g][0] & 0xFFu), s1 = e4m3_val(sc[g][0] >> 8);
               const uint32_t s02 = pack_bf16(s0, s0), s12 = pack_bf16(s1, s1);   // exact in bf16
@@ -579,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0 && ok) mbar_arrive(&ss.full_dq[j]);
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
+          for (int g = 0; g < kG; ++g) {
 #pragma unroll
             for (int jj = 0; jj + 1 < kSlabs; ++jj) { cw[g][jj] = cw[g][jj + 1]; sc[g][jj] = sc[g][jj + 1]; }
           }
@@ -598,10 +622,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ph_s ^= 1u;
       tc_fence_after();
-      const int key = qd * 32 + lane;            // this thread's key row = TMEM lane
-      bool valid;
-      if (win) {
-        const int u = (t - a.n_idx_tiles) * kTile + key;            // window slot / ring slot
+      // this thread's key row.  M = 128: TMEM lane = key.  M = 64: key m sits in lane
+      // 32 (m / 16) + m % 16, so lanes 16-31 of each quadrant hold no key ("dead": they take
+      // part in the warp's loads and reductions with p = 0 and store nothing)
+      const bool live = kT == 128 || lane < 16;
+      const int key = kT == 128 ? qd * 32 + lane : qd * 16 + (lane & 15);
+      bool valid = false;
+      if (!live) {
+      } else if (win) {
+        const int u = (t - a.n_idx_tiles) * kT + key;               // window slot / ring slot
         if (a.swa_ring) {
           // ring slot u holds the window position t_q - d, d = (t_q - u) mod ring
           const int64_t d = ((t_q - u) % a.swa_ring + a.swa_ring) % a.swa_ring;
@@ -667,8 +696,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       {
         // p = 2^(s - m_ref), rounded to bf16, written as P[head][key] (a K-major operand:
-        // two 64-key chunks of [HN rows x 128 B], 128-byte swizzle); v becomes the rounded p.
-        // An empty slot (s = -inf) gives p = 0 even while m_ref is still -inf.
+        // kT / 64 chunks of [HN rows x 64 keys x 2 B], 128-byte swizzle); v becomes the
+        // rounded p.  An empty slot (s = -inf) gives p = 0 even while m_ref is still -inf.
         uint8_t* prow = sP + (key >> 6) * G::kPChunk;
         const uint32_t unit = (uint32_t)(key & 63) >> 3, byte = (uint32_t)(key & 7) * 2;
 #pragma unroll
@@ -677,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float pe = v[e] == -INFINITY ? 0.0f : fast_exp2(v[e] - ss.m_ref[hh]);
           const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
           v[e] = __bfloat162float(pb);
-          *reinterpret_cast<__nv_bfloat16*>(prow + hh * 128 + ((unit ^ (hh & 7)) << 4) + byte) = pb;
+          if (live) *reinterpret_cast<__nv_bfloat16*>(prow + hh * 128 + ((unit ^ (hh & 7)) << 4) + byte) = pb;
         }
         warp_reduce_heads<HW, false>(v, lane);
         if (lane < HW) ss.red[qd][h0 + lane] = v[0];
@@ -814,8 +843,8 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const AttnArg
 // ---------------------------------------------------------------------------------
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int idx_tiles_of(int topk) { return (topk + kTile - 1) / kTile; }
-int win_tiles_of(int window) { return (window + kTile - 1) / kTile; }
+int idx_tiles_of(int topk, int kt) { return (topk + kt - 1) / kt; }
+int win_tiles_of(int window, int kt) { return (window + kt - 1) / kt; }
 
 int sm_count() {
   static std::atomic<int> cached[64];
@@ -838,11 +867,22 @@ int nsplit_of(int num_q, int n_tiles) {
   return std::max(1, std::min(std::min(n_tiles, kMaxSplit), per_q));
 }
 
+// Keys per tile.  64 when twice the CTAs of 128-key tiles (one per tile and group of 16
+// heads) still fit in one wave: each CTA then dequantises half the rows and issues half the
+// O MMAs (a tcgen05.mma of M = 64 costs what one of M = 128 does), which shortens a small
+// batch's chain.  128 otherwise: fewer, fuller MMAs for batches that fill the GPU.  A pure
+// function of the call's shape, so every layer of a group (and the stash) agrees.
+int tile_keys(int num_q, int H, int topk, int window) {
+  const int64_t n128 = std::max(1, idx_tiles_of(topk, 128) + win_tiles_of(window, 128));
+  const int64_t ctas = (int64_t)num_q * std::min<int64_t>(n128, kMaxSplit) * ((H + 15) / 16);
+  return 2 * ctas <= sm_count() ? 64 : 128;
+}
+
 bool attn_shape_ok(int H, int D) {
   return H >= 1 && H <= 64 && (D == 128 || D == 256 || D == 512);
 }
 
-size_t stash_tile_bytes(int D) { return (size_t)kTile * ((size_t)D / 2 + (size_t)D / 16 + 1); }
+size_t stash_tile_bytes(int D, int kt) { return (size_t)kt * ((size_t)D / 2 + (size_t)D / 16 + 1); }
 
 // the driver's tensor-map encoder, looked up once (a function-local static: thread-safe)
 PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
@@ -872,33 +912,33 @@ bool make_q_map(CUtensorMap* tm, const uint16_t* q, int num_q, int H, int D, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The window rows as a [swa_rows][D] bf16 map with boxes of 16 dims x 128 rows and the
+// The window rows as a [swa_rows][D] bf16 map with boxes of 16 dims x kt rows and the
 // 32-byte swizzle: one box is one slice of the KV tile.  Rows outside the map read as zero.
-bool make_swa_map(CUtensorMap* tm, const uint16_t* swa, int64_t rows, int D) {
+bool make_swa_map(CUtensorMap* tm, const uint16_t* swa, int64_t rows, int D, int kt) {
   auto fn = attn_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {16u, (cuuint32_t)kTile};
+  cuuint32_t box[2] = {16u, (cuuint32_t)kt};
   cuuint32_t estr[2] = {1u, 1u};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(swa), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int HN>
+template <int D, int HN, int kT>
 cudaError_t launch(AttnArgs a, const uint16_t* q, cudaStream_t st) {
-  using G = Geo<D, HN>;
+  using G = Geo<D, HN, kT>;
   CUtensorMap tm;
   if (!make_q_map(&tm, q, a.num_q, a.H, D, HN)) return checked(cudaErrorInvalidValue);
   CUtensorMap tm_swa;
   std::memset(&tm_swa, 0, sizeof(tm_swa));  // not read without window tiles
-  if (a.n_win_tiles > 0 && a.swa_rows > 0 && !make_swa_map(&tm_swa, a.swa, a.swa_rows, D))
+  if (a.n_win_tiles > 0 && a.swa_rows > 0 && !make_swa_map(&tm_swa, a.swa, a.swa_rows, D, kT))
     return checked(cudaErrorInvalidValue);
-  cudaError_t e = checked(cudaFuncSetAttribute(attn_tc_kernel<D, HN>,
+  cudaError_t e = checked(cudaFuncSetAttribute(attn_tc_kernel<D, HN, kT>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(attn_tc_kernel<D, HN>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
+  e = launch_pdl(attn_tc_kernel<D, HN, kT>, dim3(a.nsplit * a.hsplit, a.num_q), dim3(kThreads),
                  (size_t)G::kSmem, st, tm, tm_swa, a);
   if (e != cudaSuccess || a.nsplit <= 1) return e;
   return launch_pdl(attn_merge_kernel, dim3((a.H * D / 4 + kMergeThreads - 1) / kMergeThreads, a.num_q),
@@ -917,13 +957,17 @@ int heads_per_cta(int num_q, int nsplit, int H) {
 }
 
 template <int D>
-cudaError_t launch_d(AttnArgs a, const uint16_t* q, cudaStream_t st) {
+cudaError_t launch_d(AttnArgs a, const uint16_t* q, int kt, cudaStream_t st) {
+  if (kt == 64) {                                           // small batches: groups of 16 heads
+    a.hsplit = (a.H + 15) / 16;
+    return launch<D, 16, 64>(a, q, st);
+  }
   const int all = a.H <= 16 ? 16 : a.H <= 32 ? 32 : 64;     // one group of all heads
   const int g = std::min(heads_per_cta(a.num_q, a.nsplit, a.H), all);
   a.hsplit = (a.H + g - 1) / g;
-  if (g == 16) return launch<D, 16>(a, q, st);
-  if (g == 32) return launch<D, 32>(a, q, st);
-  return launch<D, 64>(a, q, st);
+  if (g == 16) return launch<D, 16, 128>(a, q, st);
+  if (g == 32) return launch<D, 32, 128>(a, q, st);
+  return launch<D, 64, 128>(a, q, st);
 }
 
 }  // namespace
@@ -933,13 +977,15 @@ using namespace csa2;
 
 extern "C" size_t csa2_sparse_attn_stash_bytes(int32_t num_q, int32_t D, int32_t topk) {
   if (num_q < 0 || D < 1 || topk < 0) return 0;
-  return (size_t)num_q * idx_tiles_of(topk) * stash_tile_bytes(D);
+  // (sized for 128-key tiles: at least what 64-key tiles of the same slots take)
+  return (size_t)num_q * idx_tiles_of(topk, kTile) * stash_tile_bytes(D, kTile);
 }
 
 extern "C" size_t csa2_sparse_attn_workspace(int32_t num_q, int32_t H, int32_t D, int32_t topk,
                                              int32_t window) {
   if (num_q < 0 || H < 1 || D < 1 || topk < 0 || window < 0) return 0;
-  const int ns = nsplit_of(num_q, idx_tiles_of(topk) + win_tiles_of(window));
+  const int kt = tile_keys(num_q, H, topk, window);
+  const int ns = nsplit_of(num_q, idx_tiles_of(topk, kt) + win_tiles_of(window, kt));
   size_t off = CSA2_STATUS_BYTES;
   if (ns > 1) {
     off = a256(off + (size_t)num_q * ns * H * D * 4);
@@ -997,13 +1043,14 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
   a.swa_ring = window > 0 ? swa_ring : 0;
   a.mode = (int)mode;
   a.stash = static_cast<uint8_t*>(kv_stash);
-  a.n_idx_tiles = idx_tiles_of(topk);
-  a.n_win_tiles = (swa_rows > 0 && window > 0) ? (a.swa_ring ? a.swa_ring / kTile : win_tiles_of(window)) : 0;
+  const int kt = tile_keys(num_q, H, topk, window);
+  a.n_idx_tiles = idx_tiles_of(topk, kt);
+  a.n_win_tiles = (swa_rows > 0 && window > 0) ? (a.swa_ring ? a.swa_ring / kt : win_tiles_of(window, kt)) : 0;
   a.H = H;
   a.scale_log2 = softmax_scale * kLog2e;
   const int n_tiles = a.n_idx_tiles + a.n_win_tiles;
   // (the split count depends on the call's shape only, as the workspace size does)
-  a.nsplit = nsplit_of(num_q, idx_tiles_of(topk) + win_tiles_of(window));
+  a.nsplit = nsplit_of(num_q, idx_tiles_of(topk, kt) + win_tiles_of(window, kt));
   a.tiles_per_split = std::max(1, (n_tiles + a.nsplit - 1) / a.nsplit);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
@@ -1016,8 +1063,8 @@ extern "C" csa2_status_t csa2_sparse_attn(const uint16_t* q, int32_t num_q, int3
 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
-  if (D == 128) e = launch_d<128>(a, q, st);
-  else if (D == 256) e = launch_d<256>(a, q, st);
-  else e = launch_d<512>(a, q, st);
+  if (D == 128) e = launch_d<128>(a, q, kt, st);
+  else if (D == 256) e = launch_d<256>(a, q, kt, st);
+  else e = launch_d<512>(a, q, kt, st);
   return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
