@@ -5,15 +5,16 @@
 // and window KV; Reuse layers attend with the latest indices) and "FP4 KV 与部署层的几个改动"
 // (E2M1 values with one E4M3 scale per 16 channels).
 //
-// The key slots of a query form 128-slot tiles: ceil(topk / 128) index tiles (the selected
-// cache rows; slots past topk are empty) and ceil(window / 128) window tiles (its window
-// positions t-W+1 .. t).  One CTA takes a contiguous range of one query's tiles for a group of
-// HN heads (the MMAs' N): 16 when a small batch leaves SMs idle (more CTAs share a query's
-// work), 32, or all 64 from a full wave on.  A tcgen05.mma of M = 128 costs about the same
-// for every N <= 64, and a CTA gathers and dequantises each of its rows once for its heads.
+// The key slots of a query form tiles of kT slots (kT = 64 for small batches, 128 once the
+// CTAs fill the GPU: tile_keys): ceil(topk / kT) index tiles (the selected cache rows; slots
+// past topk are empty) and ceil(window / kT) window tiles (its window positions t-W+1 .. t).
+// One CTA takes a contiguous range of one query's tiles for a group of HN heads (the MMAs'
+// N): 16 when a small batch leaves SMs idle (more CTAs share a query's work), 32, or all 64
+// from a full wave on.  A tcgen05.mma costs about the same for M = 64 as for M = 128 and for
+// every N <= 64, and a CTA gathers and dequantises each of its rows once for its heads.
 //
 // Warp roles (288 threads):
-//   warps 0-7  (256 threads) per index tile: thread (row r, half h) prefetches its half of
+//   warps 0-7  (256 threads) per index tile: thread (row r, quarter p) prefetches its part of
 //              row r's FP4 codes and the row's scales into registers one tile ahead (from
 //              the cache, or in a Reuse layer from the stash of the group's Full / Reindex
 //              call), then dequantises them to bf16 (exact: a 2-bit-mantissa code times a
@@ -22,7 +23,7 @@
 //              (one key per TMEM lane, half the heads per warp) writes P; at the end, O.
 //   warp 8     one thread: loads Q (TMA, once), the window tiles (TMA, one 16-dim slice per
 //              box, straight into the KV tile) and issues every MMA:
-//                S^T[key, head]  = KV[key, :] . Q[head, :]       (M = 128 keys, K = D)
+//                S^T[key, head]  = KV[key, :] . Q[head, :]       (M = kT keys, K = D)
 //                O^T[d, head]   += V^T[d, key] . P^T[key, head]  (M = 128 dims per slab)
 //              reading the same 32-byte-swizzled KV tile K-major for S^T and MN-major for O^T.
 // The slab barriers let the dequantisation of tile i+1 overlap the O MMAs of tile i, and the

@@ -278,12 +278,13 @@ CSA2_API csa2_status_t csa2_index_pool(const uint16_t* qI, const float* w, int32
  *   lse = -inf.  The two sets share one softmax; a row in both counts twice.
  * Cross-layer reuse ([SURV] §2.2.2, [MTP] "CSA2：…": a Reuse layer takes the main KV and the
  * latest Top-K of an earlier layer): with a non-NULL `kv_stash`,
- *   - mode FULL or REINDEX also stores the selected rows' FP4 codes and scales (per
- *     128-slot tile, in the kernel's staging layout) into kv_stash;
+ *   - mode FULL or REINDEX also stores the selected rows' FP4 codes and scales (per tile
+ *     of 64 or 128 slots, a choice made from num_q, H, topk and window, in the kernel's
+ *     staging layout) into kv_stash;
  *   - mode REUSE takes the selected rows from kv_stash instead of the FP4 cache.  The
  *     stash must hold the rows of exactly these indices for these queries, as written by
- *     the latest FULL/REINDEX call with the same num_q, D and topk; the window rows are
- *     always read from swa_kv.  Results equal those of a stateless call.
+ *     the latest FULL/REINDEX call with the same num_q, H, D, topk and window; the window
+ *     rows are always read from swa_kv.  Results equal those of a stateless call.
  *   With kv_stash == NULL every mode reads the FP4 cache (the call is stateless).
  *   q         device bf16 [num_q][H][D]        1 <= H <= 64, D in {128, 256, 512},
  *             num_q <= 65535 (other shapes return CSA2_ERR_UNSUPPORTED); base 16-byte
