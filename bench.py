@@ -258,11 +258,12 @@ def index_flops(W) -> int:
     return int(np.sum(W.q_visible())) * W.H_I * W.d_I * 2
 
 
-def captured_attn_traffic(workload_name: str):
+def captured_attn_traffic(workload_name: str, root: str | None = None):
     """DRAM bytes per launch of the attention kernel from the committed ncu capture
-    (profiles/attn_tc_traffic.json), or None when that capture is of another workload or
-    the kernel's sources have changed since it was taken (their SHA-256 differs)."""
-    here = os.path.dirname(os.path.abspath(__file__))
+    (profiles/attn_tc_traffic.json under ``root``, the repository by default), or None when
+    that capture is of another workload or the kernel's sources have changed since it was
+    taken (their SHA-256 differs)."""
+    here = root or os.path.dirname(os.path.abspath(__file__))
     try:
         with open(os.path.join(here, "profiles", "attn_tc_traffic.json")) as f:
             rec = json.load(f)
