@@ -734,16 +734,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     done_ok = ss.fail == 0;
     tc_fence_after();
     const bool partial = a.nsplit > 1;
-    if (done_ok) {
-      // O^T from TMEM into shared memory as [head][D] fp32 rows (the KV tile is free: every
-      // MMA has completed), then bulk copies of the H rows.  Unsplit: out = O / l.  Split:
-      // the unnormalised O (relative to m_ref) as this split's [H][D] partial, plus (m, l).
+    const int n_h = min(HN, Hr - h_lo);          // real heads of this group
+    if (done_ok && partial) {
+      // Split: the unnormalised O (relative to m_ref) as this split's [H][D] partial, written
+      // straight from TMEM (a thread holds one dim of its HW heads, so each warp store is 32
+      // consecutive dims of one head: a full 128-byte line), plus (m, l) per head.
+      float* dst = a.part_o + (((int64_t)q * a.nsplit + split) * Hr + h_lo) * D;
+#pragma unroll 1
+      for (int j = 0; j < kSlabs; ++j) {
+        const int d = j * 128 + qd * 32 + lane;
+        float o[HW];
+        if (n > 0) {
+          tmem_ld_cols<HW>(tO + lane_base + j * HN + h0, o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < HW; ++e) o[e] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < HW; ++e)
+          if (h0 + e < n_h) dst[(size_t)(h0 + e) * D + d] = o[e];
+      }
+      if (tid < n_h) {
+        const float m = ss.m_ref[tid], l = ss.l_acc[tid];
+        float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + h_lo + tid) * 2;
+        ml[0] = (n > 0 && l > 0.0f) ? m : -INFINITY;
+        ml[1] = n > 0 ? l : 0.0f;
+      }
+    } else if (done_ok) {
+      // Unsplit: out = O / l, from TMEM into shared memory as [head][D] fp32 rows (the KV
+      // tile is free: every MMA has completed), then bulk copies of the H rows.
       float* sO = reinterpret_cast<float*>(sKV);
       float osc[HW];
 #pragma unroll
       for (int e = 0; e < HW; ++e) {
         const float l = ss.l_acc[h0 + e];
-        osc[e] = n == 0 ? 0.0f : (partial ? 1.0f : (l > 0.0f ? 1.0f / l : 0.0f));
+        osc[e] = n == 0 ? 0.0f : (l > 0.0f ? 1.0f / l : 0.0f);
       }
 #pragma unroll 1
       for (int j = 0; j < kSlabs; ++j) {
@@ -760,25 +785,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       dq_sync();
-      float* dst = partial ? a.part_o + ((int64_t)q * a.nsplit + split) * Hr * D
-                           : a.out + (int64_t)q * Hr * D;
-      const int n_h = min(HN, Hr - h_lo);        // real heads of this group
+      float* dst = a.out + (int64_t)q * Hr * D;
       if (tid < 32) {
         for (int hh = tid; hh < n_h; hh += 32)
           bulk_s2g(dst + (size_t)(h_lo + hh) * D, sO + (size_t)hh * D, D * 4);
         bulk_commit();
         bulk_wait_all();
       }
-      if (tid >= 32 && tid < 32 + n_h) {
+      if (tid >= 32 && tid < 32 + n_h && a.lse) {
         const int hh = tid - 32;
         const float m = ss.m_ref[hh], l = ss.l_acc[hh];
-        if (partial) {
-          float* ml = a.part_ml + (((int64_t)q * a.nsplit + split) * Hr + h_lo + hh) * 2;
-          ml[0] = (n > 0 && l > 0.0f) ? m : -INFINITY;
-          ml[1] = n > 0 ? l : 0.0f;
-        } else if (a.lse) {
-          a.lse[(int64_t)q * Hr + h_lo + hh] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
-        }
+        a.lse[(int64_t)q * Hr + h_lo + hh] = (l > 0.0f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
     }
   }
