@@ -46,6 +46,23 @@ def test_workspace_sizes(L):
     assert csa2.sparse_attn_workspace(1, 64, 512, 512, 128) >= 256
 
 
+def test_attention_split_policy_through_workspace_sizes(L):
+    """The attention workspace holds the key splits' partials ([q][split][H][D] fp32 and
+    (m, l) [q][split][H]), so its size shows the host's tile and split choice (148 SMs
+    without a GPU).  A decode query: 64-key tiles, 8 + 2 = 10 splits; 64 queries: 128-key
+    tiles, 2 splits (SMs per query); 4,096 queries: one split, no partials."""
+    from fp4_kv_cache_03_b200 import csa2
+    sms = L.csa2_device_sms()
+    if sms > 0 and sms != 148:
+        pytest.skip(f"the expectations below are for 148 SMs, this device has {sms}")
+    a256 = lambda x: (x + 255) // 256 * 256
+    def expect(nq, ns, H=64, D=512):
+        return 256 + a256(nq * ns * H * D * 4) + a256(nq * ns * H * 2 * 4) if ns > 1 else 256
+    assert csa2.sparse_attn_workspace(1, 64, 512, 512, 128) == expect(1, 10)
+    assert csa2.sparse_attn_workspace(64, 64, 512, 512, 128) == expect(64, 2)
+    assert csa2.sparse_attn_workspace(4096, 64, 512, 512, 128) == expect(4096, 1)
+
+
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: the checks below return first
 
 
