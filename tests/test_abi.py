@@ -172,3 +172,20 @@ def test_binding_matches_header():
         params = params.strip()
         n = 0 if params in ("", "void") else len(params.split(","))
         assert len(csa2._SIGS[name][1]) == n, (name, n, len(csa2._SIGS[name][1]))
+
+
+def test_binding_rejects_wrong_dtypes_before_any_call(L):
+    """The binding checks tensor dtypes before it calls into the library (a wrong dtype would
+    otherwise reach a kernel as a mis-sized buffer); CPU tensors suffice: nothing runs."""
+    import torch
+    from fp4_kv_cache_03_b200 import csa2
+    qI = torch.zeros(1, 16, 128, dtype=torch.bfloat16)
+    idx_k = torch.zeros(256, 128, dtype=torch.bfloat16)
+    seqs = csa2.Seqs(1, 1, FAKE, FAKE)
+    good_w = torch.zeros(1, 16, dtype=torch.float32)
+    good_i = torch.zeros(1, 64, dtype=torch.int32)
+    for w, ind, pool in [(good_w.double(), good_i, None), (good_w, good_i.long(), None),
+                         (good_w, good_i, torch.zeros(1, 8, dtype=torch.int64))]:
+        with pytest.raises(AssertionError):
+            csa2.index_full_noalloc(qI, w, idx_k, seqs, 64, ind, 256, pool_blocks=8 if pool is not None else 0,
+                                    pool=pool)
